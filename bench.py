@@ -1,0 +1,494 @@
+#!/usr/bin/env python
+"""Benchmark of librlscan: env-steps/s per estimator and fraction of the B200
+HBM roofline, on the sequence-length sweep N = 4096, T = 32..2048.
+
+One *step* is one pass of the whole hot path over one batch of synthetic
+rollouts: every estimator of the workload at every T of the sweep (the
+default workload: GAE, V-trace, TD(lambda) and discounted returns at
+T = 32, 64, ..., 2048 with per-step truncation -- 28 fused kernel launches).
+Inputs are resident in HBM before the timed region; every call reads its own
+buffers, so a step touches ~1.1 GB of distinct inputs (8.5x the 126 MB L2)
+and no call finds its inputs in L2.  Steps are replayed from CUDA graphs;
+timing-event nodes between launches give each kernel's duration on the
+launching stream.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+        python bench.py --impl reference ...     (the fp64 CPU oracle, timed)
+Under torchrun each rank processes its own rollout shard of the workload
+(weak scaling, no data-path collective); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from segmented_linear_recurrence_b200 import synthetic  # noqa: E402
+
+METRIC = "env-steps/sec per estimator and % of B200 HBM roofline, N=4096, T=32..2048"
+UNIT = "env-steps/s"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+DEFAULT_WORKLOAD = "sweep_4096xT"
+
+# Bytes per env-step each estimator must move at minimum (mandatory inputs
+# read once, outputs written once): fp32/int32 = 4 B, flags = 1 B.
+def algorithmic_bytes(est: str, d: dict) -> int:
+    """Strict algorithmic HBM bytes of one call on inputs `d`.
+
+    Per-step arrays count their full size; `truncated` adds its flag bytes and
+    `trunc_value` is counted only where truncated (one 32-byte sector each);
+    per-row arrays (bootstrap, init_trace) count 4 B per row; every output
+    counts 4 B per step."""
+    if est == "retrace":
+        N, T, A = d["q"].shape
+    else:
+        key = {"elig_trace": "inputs", "episodic_prefix_sum": "x"}.get(est, "rewards")
+        N, T = d[key].shape
+        A = 0
+    nt = N * T
+    per_step_in = {
+        "gae": ("rewards", "values"), "td_lambda": ("rewards", "values"),
+        "vtrace": ("log_rhos", "rewards", "values"), "discounted_return": ("rewards",),
+        "elig_trace": ("inputs",), "episodic_prefix_sum": ("x",),
+        "retrace": ("mu_a", "actions", "rewards"),
+    }[est]
+    b = sum(4 * nt for k in per_step_in)
+    if est == "retrace":
+        b += 2 * 4 * nt * A  # q and pi
+    if d.get("terminated") is not None:
+        b += nt
+    if d.get("truncated") is not None:
+        b += nt
+        if d.get("trunc_value") is not None:
+            b += 32 * int(np.count_nonzero(d["truncated"]))
+    for k in ("bootstrap", "init_trace"):
+        if d.get(k) is not None:
+            b += 4 * N
+    n_out = {"gae": 2, "vtrace": 2}.get(est, 1)
+    b += 4 * nt * n_out
+    return int(b)
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def load_traffic(kernel_key: str):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summary, if it
+    was taken on the current kernel sources (else None)."""
+    from segmented_linear_recurrence_b200 import build as slr_build
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+    except Exception:
+        return None
+    if j.get("source_hash") != slr_build.source_hash():
+        return None
+    k = j.get("kernels", {}).get(kernel_key)
+    return None if k is None else k.get("dram_bytes_per_full_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", gpu_id],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+ARG_ORDER = {
+    "gae": ("rewards", "values", "bootstrap", "terminated", "truncated", "trunc_value"),
+    "vtrace": ("log_rhos", "rewards", "values", "bootstrap", "terminated", "truncated", "trunc_value"),
+    "retrace": ("q", "pi", "mu_a", "actions", "rewards", "bootstrap", "terminated", "truncated",
+                "trunc_value"),
+    "td_lambda": ("rewards", "values", "bootstrap", "terminated", "truncated", "trunc_value"),
+    "discounted_return": ("rewards", "bootstrap", "terminated", "truncated", "trunc_value"),
+    "elig_trace": ("inputs", "init_trace", "terminated", "truncated"),
+    "episodic_prefix_sum": ("x", "terminated", "truncated"),
+}
+OUT_KW = {"gae": ("advantages", "returns"), "vtrace": ("vs", "pg_advantages"), "retrace": ("q_ret",),
+          "td_lambda": ("returns",), "discounted_return": ("returns",), "elig_trace": ("traces",),
+          "episodic_prefix_sum": ("out",)}
+
+
+def workload_calls(workload: str, rank: int):
+    """Host inputs of every call of one step: list of (est, T, dict)."""
+    w = synthetic.WORKLOADS[workload]
+    calls = []
+    for est in w["estimators"]:
+        for T in w["Ts"]:
+            seed = synthetic.seed_for(workload, est, T) + 7919 * rank
+            d = synthetic.make_inputs(est, w["N"], T, seed=seed, p_term=w["p_term"],
+                                      p_trunc=w["p_trunc"], A=w.get("A", 18))
+            calls.append((est, T, d))
+    return calls
+
+
+class DeviceCall:
+    def __init__(self, est, T, d, device):
+        import torch
+        self.est, self.T = est, T
+        self.inputs = [None if d.get(k) is None else torch.from_numpy(d[k]).to(device)
+                       for k in ARG_ORDER[est]]
+        shape = d["q"].shape[:2] if est == "retrace" else d[ARG_ORDER[est][0]].shape
+        dt = torch.int32 if est == "episodic_prefix_sum" else torch.float32
+        self.outs = {k: torch.empty(tuple(shape), dtype=dt, device=device) for k in OUT_KW[est]}
+        self.scal = {} if est == "episodic_prefix_sum" else dict(synthetic.SCALARS[est])
+        self.steps = int(np.prod(shape))
+        self.bytes = algorithmic_bytes(est, d)
+
+    def launch(self):
+        import segmented_linear_recurrence_b200 as slr
+        getattr(slr, f"rlscan_{self.est}")(*self.inputs, **self.scal, **self.outs)
+
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import segmented_linear_recurrence_b200 as slr
+    from segmented_linear_recurrence_b200 import build as slr_build
+
+    slr_build.build()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+
+    host_calls = workload_calls(args.workload, rank)
+    calls = [DeviceCall(est, T, d, device) for est, T, d in host_calls]
+    steps_per_step = sum(c.steps for c in calls)
+    launches_per_step = 0
+    for est, T, d in host_calls:
+        A = d["q"].shape[2] if est == "retrace" else 1
+        N = d["q"].shape[0] if est == "retrace" else d[ARG_ORDER[est][0]].shape[0]
+        launches_per_step += slr.rlscan_query_plan(est, N, T, A)["launches"]
+
+    def eager_step():
+        for c in calls:
+            c.launch()
+
+    # warm-up: one eager step (allocates any look-back workspace), then graphs
+    warm_done = 0
+    eager_step()
+    warm_done += 1
+    torch.cuda.synchronize()
+    if slr.rlscan_sync_status() != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    P = max(1, min(args.steps, 8))
+    graphs, events = [], []
+    for _ in range(P):
+        g = torch.cuda.CUDAGraph()
+        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
+        with torch.cuda.graph(g, stream=torch.cuda.Stream(device)):
+            cur = torch.cuda.current_stream()
+            evs[0].record(cur)
+            for j, c in enumerate(calls):
+                c.launch()
+                evs[j + 1].record(cur)
+        graphs.append(g)
+        events.append(evs)
+    while warm_done < max(args.warmup, 1):
+        graphs[warm_done % P].replay()
+        warm_done += 1
+    torch.cuda.synchronize()
+
+    gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    sampler = ClockSampler(gpu_uuid)
+    time.sleep(0.3)  # let the sampler start before the timed region
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(args.steps):
+        graphs[k % P].replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    elapsed_ms = t0.elapsed_time(t1)
+    status = slr.rlscan_sync_status()
+
+    # per-launch durations (last replay of each graph in the timed region)
+    per_call_ms = np.zeros(len(calls))
+    for evs in events:
+        for j in range(len(calls)):
+            per_call_ms[j] += evs[j].elapsed_time(evs[j + 1])
+    per_call_ms /= P
+
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+
+    # e2e: the same step through the public API from pinned host buffers
+    e2e = run_e2e(args, host_calls, device, world)
+
+    return dict(calls=calls, steps_per_step=steps_per_step, launches_per_step=launches_per_step,
+                elapsed_ms=max_ms, per_call_ms=per_call_ms, clocks=clocks, e2e=e2e,
+                warmup=warm_done, status=status)
+
+
+def run_e2e(args, host_calls, device, world):
+    import torch
+    import torch.distributed as dist
+
+    import segmented_linear_recurrence_b200 as slr
+    pinned = []
+    h2d = d2h = 0
+    for est, T, d in host_calls:
+        ins = [None if d.get(k) is None else torch.from_numpy(d[k]).pin_memory() for k in ARG_ORDER[est]]
+        h2d += sum(x.numel() * x.element_size() for x in ins if x is not None)
+        shape = d["q"].shape[:2] if est == "retrace" else d[ARG_ORDER[est][0]].shape
+        d2h += 4 * int(np.prod(shape)) * len(OUT_KW[est])
+        scal = {} if est == "episodic_prefix_sum" else dict(synthetic.SCALARS[est])
+        pinned.append((est, ins, scal))
+
+    def step():
+        out = None
+        for est, ins, scal in pinned:
+            out = getattr(slr, f"rlscan_{est}")(*ins, **scal)
+        return out
+
+    step()  # warm the caching allocators
+    torch.cuda.synchronize()
+    n = max(1, args.e2e_steps)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(n):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    return dict(ms_per_step=float(ms.item()) / n, steps=n, h2d=h2d, d2h=d2h)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline / reference arm)
+# ---------------------------------------------------------------------------
+def oracle_pass(host_calls):
+    import oracle
+    steps = 0
+    for est, T, d in host_calls:
+        oracle.run(est, d, **synthetic.SCALARS[est])
+        steps += d["q"].shape[0] * d["q"].shape[1] if est == "retrace" else int(np.prod(
+            d[ARG_ORDER[est][0]].shape))
+    return steps
+
+
+def cpu_baseline(host_calls, seconds: float):
+    """Times the oracle (single-threaded plain C loops) over whole passes of
+    the workload until at least `seconds` of CPU work has run."""
+    oracle_pass([host_calls[0]])  # build / load
+    done_steps, passes = 0, 0
+    t0 = time.perf_counter()
+    while True:
+        done_steps += oracle_pass(host_calls)
+        passes += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done_steps / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{passes} full pass(es) over the workload ({done_steps} env-steps, "
+                      f"{dt:.1f} s, one thread, fp64)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    host_calls = workload_calls(args.workload, 0)
+    per_pass = oracle_pass([host_calls[0]])  # build / load
+    for _ in range(max(args.warmup, 0)):
+        oracle_pass(host_calls)
+    t0 = time.perf_counter()
+    steps = 0
+    for _ in range(args.steps):
+        steps += oracle_pass(host_calls)
+    dt = time.perf_counter() - t0
+    value = steps / dt
+    cores = 1
+    w = synthetic.WORKLOADS[args.workload]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": int(os.environ.get("WORLD_SIZE", args.gpus)), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * dt / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "estimators": list(w["estimators"]), "N_envs": w["N"],
+                   "T": list(w["Ts"]), "implementation": "fp64 sequential CPU oracle (oracle/)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{args.steps} full pass(es) over the workload, one thread"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    del per_pass
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=tuple(synthetic.WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU work for the oracle baseline (0 disables it)")
+    args = ap.parse_args()
+
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    res = run_gpu(args, rank, world, local_rank)
+
+    calls = res["calls"]
+    ms_step = res["elapsed_ms"] / args.steps
+    value = world * res["steps_per_step"] / (ms_step / 1000.0)
+    peak, peak_kind = measured_peak()
+
+    # per-estimator breakdown and the dominant kernel
+    per_est = {}
+    for c, ms in zip(calls, res["per_call_ms"]):
+        e = per_est.setdefault(c.est, {"ms": 0.0, "bytes": 0, "launches": 0, "by_T": {}})
+        e["ms"] += ms
+        e["bytes"] += c.bytes
+        e["launches"] += 1
+        gbs = c.bytes / (ms / 1000.0) / 1e9
+        e["by_T"][str(c.T)] = {"us": round(ms * 1000.0, 2),
+                               "gsteps_s": round(c.steps / (ms / 1000.0) / 1e9, 2),
+                               "gbs": round(gbs, 1), "frac_of_measured": round(gbs / peak, 3),
+                               "frac_of_8TBs": round(gbs / SPEC_HBM_GBS, 3)}
+    dom = max(per_est, key=lambda k: per_est[k]["ms"])
+    de = per_est[dom]
+    achieved = de["bytes"] / (de["ms"] / 1000.0) / 1e9
+    dom_kernel = f"scan_kernel<{dom}>"
+    traffic = load_traffic(dom)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "kernel": dom_kernel, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                "algorithmic_bytes_per_launch": int(de["bytes"] / de["launches"]),
+                "avg_launch_us": round(1000.0 * de["ms"] / de["launches"], 2),
+                "frac_of_8TBs_spec": round(achieved / SPEC_HBM_GBS, 4)}
+
+    e2e = res["e2e"]
+    e2e_value = world * res["steps_per_step"] / (e2e["ms_per_step"] / 1000.0)
+
+    w = synthetic.WORKLOADS[args.workload]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": res["warmup"], "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": args.workload, "estimators": list(w["estimators"]),
+                   "N_envs_per_gpu": w["N"], "T": list(w["Ts"]), "p_term": w["p_term"],
+                   "p_trunc": w["p_trunc"], "calls_per_step": len(calls),
+                   "l2": "inputs > L2: every call reads its own buffers; "
+                         f"{sum(sum(x.numel() * x.element_size() for x in c.inputs if x is not None) for c in calls) / 1e9:.2f}"
+                         " GB of distinct inputs per step",
+                   "timing": "CUDA-graph replay of each step; timing-event nodes between launches",
+                   "parallelism": f"dp{world} (independent env shards, no collective)"},
+        "roofline": roofline,
+        "gpu_launches": int(res["launches_per_step"] * args.steps),
+        "clocks": res["clocks"],
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(e2e["h2d"]),
+                "d2h_bytes_per_step": int(e2e["d2h"]), "ms_per_step": e2e["ms_per_step"],
+                "steps": e2e["steps"], "path": "public Python API on pinned host tensors"},
+        "per_estimator": {k: {"gbs": round(v["bytes"] / (v["ms"] / 1000.0) / 1e9, 1),
+                              "frac_of_measured": round(v["bytes"] / (v["ms"] / 1000.0) / 1e9 / peak, 4),
+                              "by_T": v["by_T"]} for k, v in per_est.items()},
+        "device_status": res["status"],
+    }
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        line["cpu_baseline"] = cpu_baseline(workload_calls(args.workload, 0), args.cpu_seconds)
+    elif rank == 0:
+        line["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

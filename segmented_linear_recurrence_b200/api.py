@@ -1,1 +1,346 @@
-__all__ = []
+"""Python binding of librlscan: torch tensors in, the C ABI of ``include/rlscan.h`` underneath.
+
+Every function here only marshals arguments: it checks dtypes and shapes,
+allocates missing outputs with torch, passes raw device pointers and the
+current CUDA stream to the same-named ``extern "C"`` entry point, and turns a
+non-OK status into :class:`RlscanError`.  All arithmetic runs in the CUDA
+kernels of ``librlscan.so``; there is no CPU fallback -- if the library is
+missing or no GPU is present, the call raises.
+
+Host (CPU) tensors are accepted too: they are copied to the current CUDA
+device on the current stream, the kernel runs there, and the outputs are
+copied back into (pinned, when the inputs were pinned) host tensors.  Use
+pinned inputs for asynchronous copies.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "RlscanError", "lib", "rlscan_gae", "rlscan_vtrace", "rlscan_retrace", "rlscan_td_lambda",
+    "rlscan_discounted_return", "rlscan_elig_trace", "rlscan_episodic_prefix_sum",
+    "rlscan_sync_status", "rlscan_status_string", "rlscan_release_workspaces",
+    "rlscan_abi_version", "rlscan_query_plan", "rlscan_set_option", "rlscan_get_option",
+    "STATUS", "OPTIONS", "ESTIMATOR_IDS", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librlscan.so")
+
+STATUS = {0: "RLSCAN_OK", 1: "RLSCAN_ERR_INVALID_ARG", 2: "RLSCAN_ERR_OVERLAP",
+          3: "RLSCAN_ERR_LAUNCH", 4: "RLSCAN_ERR_TIMEOUT", 5: "RLSCAN_ERR_NOMEM",
+          6: "RLSCAN_ERR_CUDA", 7: "RLSCAN_ERR_CAPTURE"}
+OPTIONS = {"lookback_timeout_ns": 1, "force_lookback": 2, "force_block": 3, "force_scalar": 4,
+           "check_pointers": 5, "test_starve_lookback": 6}
+ESTIMATOR_IDS = {"gae": 0, "vtrace": 1, "retrace": 2, "td_lambda": 3, "discounted_return": 4,
+                 "elig_trace": 5, "episodic_prefix_sum": 6}
+
+
+class RlscanError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = int(status)
+        super().__init__(f"{fn} failed: {STATUS.get(self.status, self.status)}")
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("block_threads", ctypes.c_int32), ("chunk_steps", ctypes.c_int32),
+                ("lookback", ctypes.c_int32), ("launches", ctypes.c_int32),
+                ("blocks", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
+
+
+_lib = None
+_VP, _I64, _F, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int
+_SIGNATURES = {
+    "rlscan_gae": [_VP] * 8 + [_I64, _I64, _F, _F, _VP],
+    "rlscan_vtrace": [_VP] * 9 + [_I64, _I64, _F, _F, _F, _F, _VP],
+    "rlscan_retrace": [_VP] * 10 + [_I64, _I64, _I64, _F, _F, _VP],
+    "rlscan_td_lambda": [_VP] * 7 + [_I64, _I64, _F, _F, _VP],
+    "rlscan_discounted_return": [_VP] * 6 + [_I64, _I64, _F, _VP],
+    "rlscan_elig_trace": [_VP] * 5 + [_I64, _I64, _F, _F, _VP],
+    "rlscan_episodic_prefix_sum": [_VP] * 4 + [_I64, _I64, _VP],
+    "rlscan_sync_status": [_VP],
+    "rlscan_release_workspaces": [],
+    "rlscan_abi_version": [],
+    "rlscan_query_plan": [_I, _I64, _I64, _I64, ctypes.POINTER(PlanInfo)],
+    "rlscan_set_option": [_I, _I64],
+    "rlscan_get_option": [_I],
+    "rlscan_status_string": [_I],
+}
+
+
+def lib():
+    """The loaded librlscan (ctypes), with argument types declared.
+
+    Raises RuntimeError if the shared library has not been built: there is
+    no other implementation to fall back to."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"librlscan.so is missing ({LIB_PATH}); build it with "
+                               "`python -m segmented_linear_recurrence_b200.build`")
+        cdll = ctypes.CDLL(LIB_PATH)
+        for name, argtypes in _SIGNATURES.items():
+            fn = getattr(cdll, name)
+            fn.argtypes = argtypes
+            fn.restype = ctypes.c_int
+        cdll.rlscan_status_string.restype = ctypes.c_char_p
+        cdll.rlscan_get_option.restype = ctypes.c_int64
+        cdll.rlscan_release_workspaces.restype = None
+        _lib = cdll
+    return _lib
+
+
+# ---------------------------------------------------------------------------
+# marshalling helpers
+# ---------------------------------------------------------------------------
+
+class _Call:
+    """Collects the device tensors of one call; moves host tensors to the GPU."""
+
+    def __init__(self, name, ref):
+        self.name = name
+        if ref.is_cuda:
+            self.device = ref.device
+            self.host = False
+        else:
+            if not torch.cuda.is_available():
+                raise RuntimeError(f"{name}: librlscan needs a CUDA device")
+            self.device = torch.device("cuda", torch.cuda.current_device())
+            self.host = True
+            self.pinned = ref.is_pinned()
+        self.keep = []
+
+    def tensor(self, x, dtype, shape, what, required=True):
+        if x is None:
+            if required:
+                raise ValueError(f"{self.name}: {what} is required")
+            return None
+        if not isinstance(x, torch.Tensor):
+            raise TypeError(f"{self.name}: {what} must be a torch.Tensor")
+        if x.dtype != dtype and not (dtype == torch.uint8 and x.dtype == torch.bool):
+            raise TypeError(f"{self.name}: {what} must be {dtype}, got {x.dtype}")
+        if tuple(x.shape) != tuple(shape):
+            raise ValueError(f"{self.name}: {what} must have shape {tuple(shape)}, got {tuple(x.shape)}")
+        if self.host:
+            if x.is_cuda:
+                raise ValueError(f"{self.name}: mix of host and device tensors")
+            x = x.to(self.device, non_blocking=True)
+        elif x.device != self.device:
+            raise ValueError(f"{self.name}: {what} is on {x.device}, expected {self.device}")
+        if not x.is_contiguous():
+            raise ValueError(f"{self.name}: {what} must be contiguous")
+        self.keep.append(x)
+        return x
+
+    def output(self, x, dtype, shape, what):
+        if x is None:
+            x = torch.empty(shape, dtype=dtype, device=self.device)
+        elif self.host:
+            raise ValueError(f"{self.name}: pass no {what} buffer when the inputs are host tensors")
+        else:
+            self.tensor(x, dtype, shape, what)
+        self.keep.append(x)
+        return x
+
+    @staticmethod
+    def ptr(x):
+        return None if x is None else ctypes.c_void_p(x.data_ptr())
+
+    def stream(self, stream):
+        s = torch.cuda.current_stream(self.device) if stream is None else stream
+        return ctypes.c_void_p(s.cuda_stream)
+
+    def finish(self, status, outs):
+        if status != 0:
+            raise RlscanError(self.name, status)
+        if not self.host:
+            return outs
+        res = []
+        for o in outs:
+            if o is None:
+                res.append(None)
+                continue
+            h = torch.empty(o.shape, dtype=o.dtype, pin_memory=self.pinned)
+            h.copy_(o, non_blocking=self.pinned)
+            res.append(h)
+        if self.pinned:
+            torch.cuda.current_stream(self.device).synchronize()
+        return tuple(res)
+
+
+def _nt(x, name):
+    if not isinstance(x, torch.Tensor) or x.dim() != 2:
+        raise ValueError(f"{name}: per-step inputs must be 2-D [N, T] tensors")
+    return int(x.shape[0]), int(x.shape[1])
+
+
+# ---------------------------------------------------------------------------
+# estimators
+# ---------------------------------------------------------------------------
+
+def rlscan_gae(rewards, values, bootstrap, terminated=None, truncated=None, trunc_value=None, *,
+               gamma=0.99, lam=0.95, advantages=None, returns=None, want_returns=True, stream=None):
+    """GAE advantages and returns.  Returns (advantages, returns or None)."""
+    N, T = _nt(rewards, "rlscan_gae")
+    c = _Call("rlscan_gae", rewards)
+    r = c.tensor(rewards, torch.float32, (N, T), "rewards")
+    v = c.tensor(values, torch.float32, (N, T), "values")
+    b = c.tensor(bootstrap, torch.float32, (N,), "bootstrap")
+    te = c.tensor(terminated, torch.uint8, (N, T), "terminated", required=False)
+    tr = c.tensor(truncated, torch.uint8, (N, T), "truncated", required=False)
+    tv = c.tensor(trunc_value, torch.float32, (N, T), "trunc_value", required=tr is not None)
+    adv = c.output(advantages, torch.float32, (N, T), "advantages")
+    ret = c.output(returns, torch.float32, (N, T), "returns") if (want_returns or returns is not None) else None
+    st = lib().rlscan_gae(c.ptr(r), c.ptr(v), c.ptr(b), c.ptr(te), c.ptr(tr), c.ptr(tv), c.ptr(adv),
+                          c.ptr(ret), N, T, float(gamma), float(lam), c.stream(stream))
+    return c.finish(st, (adv, ret))
+
+
+def rlscan_vtrace(log_rhos, rewards, values, bootstrap, terminated=None, truncated=None,
+                  trunc_value=None, *, gamma=0.99, lam=1.0, rho_bar=1.0, c_bar=1.0, vs=None,
+                  pg_advantages=None, want_pg=True, stream=None):
+    """V-trace targets vs and policy-gradient advantages.  Returns (vs, pg or None)."""
+    N, T = _nt(rewards, "rlscan_vtrace")
+    c = _Call("rlscan_vtrace", rewards)
+    lr = c.tensor(log_rhos, torch.float32, (N, T), "log_rhos")
+    r = c.tensor(rewards, torch.float32, (N, T), "rewards")
+    v = c.tensor(values, torch.float32, (N, T), "values")
+    b = c.tensor(bootstrap, torch.float32, (N,), "bootstrap")
+    te = c.tensor(terminated, torch.uint8, (N, T), "terminated", required=False)
+    tr = c.tensor(truncated, torch.uint8, (N, T), "truncated", required=False)
+    tv = c.tensor(trunc_value, torch.float32, (N, T), "trunc_value", required=tr is not None)
+    out_vs = c.output(vs, torch.float32, (N, T), "vs")
+    pg = c.output(pg_advantages, torch.float32, (N, T), "pg_advantages") if (want_pg or pg_advantages is not None) else None
+    st = lib().rlscan_vtrace(c.ptr(lr), c.ptr(r), c.ptr(v), c.ptr(b), c.ptr(te), c.ptr(tr), c.ptr(tv),
+                             c.ptr(out_vs), c.ptr(pg), N, T, float(gamma), float(lam),
+                             float(rho_bar), float(c_bar), c.stream(stream))
+    return c.finish(st, (out_vs, pg))
+
+
+def rlscan_retrace(q, pi, mu_a, actions, rewards, bootstrap, terminated=None, truncated=None,
+                   trunc_value=None, *, gamma=0.99, lam=0.95, q_ret=None, stream=None):
+    """Retrace(lambda) targets for the taken actions.  Returns q_ret."""
+    if not isinstance(q, torch.Tensor) or q.dim() != 3:
+        raise ValueError("rlscan_retrace: q must be a 3-D [N, T, A] tensor")
+    N, T, A = (int(s) for s in q.shape)
+    c = _Call("rlscan_retrace", q)
+    qq = c.tensor(q, torch.float32, (N, T, A), "q")
+    pp = c.tensor(pi, torch.float32, (N, T, A), "pi")
+    mu = c.tensor(mu_a, torch.float32, (N, T), "mu_a")
+    ac = c.tensor(actions, torch.int32, (N, T), "actions")
+    r = c.tensor(rewards, torch.float32, (N, T), "rewards")
+    b = c.tensor(bootstrap, torch.float32, (N,), "bootstrap")
+    te = c.tensor(terminated, torch.uint8, (N, T), "terminated", required=False)
+    tr = c.tensor(truncated, torch.uint8, (N, T), "truncated", required=False)
+    tv = c.tensor(trunc_value, torch.float32, (N, T), "trunc_value", required=tr is not None)
+    out = c.output(q_ret, torch.float32, (N, T), "q_ret")
+    st = lib().rlscan_retrace(c.ptr(qq), c.ptr(pp), c.ptr(mu), c.ptr(ac), c.ptr(r), c.ptr(b), c.ptr(te),
+                              c.ptr(tr), c.ptr(tv), c.ptr(out), N, T, A, float(gamma), float(lam),
+                              c.stream(stream))
+    return c.finish(st, (out,))[0]
+
+
+def rlscan_td_lambda(rewards, values, bootstrap, terminated=None, truncated=None, trunc_value=None,
+                     *, gamma=0.99, lam=0.95, returns=None, stream=None):
+    """TD(lambda) returns.  Returns the [N, T] returns."""
+    N, T = _nt(rewards, "rlscan_td_lambda")
+    c = _Call("rlscan_td_lambda", rewards)
+    r = c.tensor(rewards, torch.float32, (N, T), "rewards")
+    v = c.tensor(values, torch.float32, (N, T), "values")
+    b = c.tensor(bootstrap, torch.float32, (N,), "bootstrap")
+    te = c.tensor(terminated, torch.uint8, (N, T), "terminated", required=False)
+    tr = c.tensor(truncated, torch.uint8, (N, T), "truncated", required=False)
+    tv = c.tensor(trunc_value, torch.float32, (N, T), "trunc_value", required=tr is not None)
+    out = c.output(returns, torch.float32, (N, T), "returns")
+    st = lib().rlscan_td_lambda(c.ptr(r), c.ptr(v), c.ptr(b), c.ptr(te), c.ptr(tr), c.ptr(tv), c.ptr(out),
+                                N, T, float(gamma), float(lam), c.stream(stream))
+    return c.finish(st, (out,))[0]
+
+
+def rlscan_discounted_return(rewards, bootstrap=None, terminated=None, truncated=None,
+                             trunc_value=None, *, gamma=0.99, returns=None, stream=None):
+    """Discounted returns (bootstrap optional).  Returns the [N, T] returns."""
+    N, T = _nt(rewards, "rlscan_discounted_return")
+    c = _Call("rlscan_discounted_return", rewards)
+    r = c.tensor(rewards, torch.float32, (N, T), "rewards")
+    b = c.tensor(bootstrap, torch.float32, (N,), "bootstrap", required=False)
+    te = c.tensor(terminated, torch.uint8, (N, T), "terminated", required=False)
+    tr = c.tensor(truncated, torch.uint8, (N, T), "truncated", required=False)
+    tv = c.tensor(trunc_value, torch.float32, (N, T), "trunc_value", required=tr is not None)
+    out = c.output(returns, torch.float32, (N, T), "returns")
+    st = lib().rlscan_discounted_return(c.ptr(r), c.ptr(b), c.ptr(te), c.ptr(tr), c.ptr(tv), c.ptr(out),
+                                        N, T, float(gamma), c.stream(stream))
+    return c.finish(st, (out,))[0]
+
+
+def rlscan_elig_trace(inputs, init_trace=None, terminated=None, truncated=None, *, gamma=0.99,
+                      lam=0.95, traces=None, stream=None):
+    """Accumulating eligibility traces (forward in time).  Returns the [N, T] traces."""
+    N, T = _nt(inputs, "rlscan_elig_trace")
+    c = _Call("rlscan_elig_trace", inputs)
+    g = c.tensor(inputs, torch.float32, (N, T), "inputs")
+    e0 = c.tensor(init_trace, torch.float32, (N,), "init_trace", required=False)
+    te = c.tensor(terminated, torch.uint8, (N, T), "terminated", required=False)
+    tr = c.tensor(truncated, torch.uint8, (N, T), "truncated", required=False)
+    out = c.output(traces, torch.float32, (N, T), "traces")
+    st = lib().rlscan_elig_trace(c.ptr(g), c.ptr(e0), c.ptr(te), c.ptr(tr), c.ptr(out), N, T,
+                                 float(gamma), float(lam), c.stream(stream))
+    return c.finish(st, (out,))[0]
+
+
+def rlscan_episodic_prefix_sum(x, terminated=None, truncated=None, *, out=None, stream=None):
+    """Episodic inclusive prefix sums of int32 values.  Returns the [N, T] int32 sums."""
+    N, T = _nt(x, "rlscan_episodic_prefix_sum")
+    c = _Call("rlscan_episodic_prefix_sum", x)
+    xx = c.tensor(x, torch.int32, (N, T), "x")
+    te = c.tensor(terminated, torch.uint8, (N, T), "terminated", required=False)
+    tr = c.tensor(truncated, torch.uint8, (N, T), "truncated", required=False)
+    o = c.output(out, torch.int32, (N, T), "out")
+    st = lib().rlscan_episodic_prefix_sum(c.ptr(xx), c.ptr(te), c.ptr(tr), c.ptr(o), N, T,
+                                          c.stream(stream))
+    return c.finish(st, (o,))[0]
+
+
+# ---------------------------------------------------------------------------
+# status, options, plans
+# ---------------------------------------------------------------------------
+
+def rlscan_sync_status(stream=None, raise_on_error=False):
+    """Synchronize the stream and return (and clear) the device-side status code."""
+    s = torch.cuda.current_stream() if stream is None else stream
+    st = int(lib().rlscan_sync_status(ctypes.c_void_p(s.cuda_stream)))
+    if raise_on_error and st != 0:
+        raise RlscanError("rlscan_sync_status", st)
+    return st
+
+
+def rlscan_status_string(status: int) -> str:
+    return lib().rlscan_status_string(int(status)).decode()
+
+
+def rlscan_release_workspaces():
+    lib().rlscan_release_workspaces()
+
+
+def rlscan_abi_version() -> int:
+    return int(lib().rlscan_abi_version())
+
+
+def rlscan_query_plan(estimator: str, N: int, T: int, A: int = 1) -> dict:
+    info = PlanInfo()
+    st = lib().rlscan_query_plan(ESTIMATOR_IDS[estimator], int(N), int(T), int(A), ctypes.byref(info))
+    if st != 0:
+        raise RlscanError("rlscan_query_plan", st)
+    return {f: getattr(info, f) for f, _ in PlanInfo._fields_}
+
+
+def rlscan_set_option(name: str, value: int):
+    st = lib().rlscan_set_option(OPTIONS[name], int(value))
+    if st != 0:
+        raise RlscanError("rlscan_set_option", st)
+
+
+def rlscan_get_option(name: str) -> int:
+    return int(lib().rlscan_get_option(OPTIONS[name]))

@@ -1,0 +1,277 @@
+// retrace.cuh -- Retrace(lambda) coefficient builder with an on-chip reduction
+// of E_pi Q over the action dimension.
+//
+// "rl-triton: High-Performance Triton GPU Kernels for Reinforcement Learning
+// Credit Assignment" (gist.science technical summary), Resultaten: Retrace is
+// the estimator with the heaviest per-step work (it loads the action
+// probabilities) and, in the pages' row-per-program design, runs short of
+// registers beyond T = 2048.  Here the per-step action rows never sit in
+// registers: each block stages its chunk's q and pi rows in shared memory
+// with TMA bulk copies (cp.async.bulk, completion on an mbarrier, no
+// multicast), a ring of `stages` sub-tiles deep, and reduces each step's row
+// to three scalars -- E_t = sum_a pi[t,a] q[t,a], q_t = q[t, a_t] and
+// c_t = lambda min(1, pi[t, a_t] / mu_t) -- kept in shared memory for the scan
+// (Munos et al. 2016).  Step t's coefficients read those of step t+1 only:
+//   a_t = gamma c_{t+1} cont_t,
+//   b_t = r_t + gamma cont_t (E_{t+1} - c_{t+1} q_{t+1}) + gamma (1 - cont_t) nv_t.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "estimators.cuh"
+#include "scan_core.cuh"
+
+namespace rlscan {
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Global -> shared bulk copy (no tensor map, no multicast); `bytes` is a
+// multiple of 16 and both addresses are 16-byte aligned.
+__device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes,
+                                              uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Bounded wait for an mbarrier phase: gives up after `timeout_ns` of global
+// time, recording the timeout status (the block then carries on with whatever
+// the buffer holds, so it neither hangs nor traps).
+__device__ __forceinline__ void mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  uint64_t timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = global_timer_ns();
+  uint64_t iters = 0;
+  const uint64_t max_iters = 64 + timeout_ns / 16;
+  while (!mbar_try_wait(bar, parity)) {
+    if (++iters > max_iters || global_timer_ns() - t0 > timeout_ns) {
+      record_status(kDevStatusTimeout);
+      return;
+    }
+  }
+}
+
+struct RetraceOp {
+  using V = float;
+  static constexpr bool kBackward = true, kNeedsNbr = true, kPrologue = true;
+  struct Args {
+    const float *q, *pi, *mu, *r, *boot, *tv;
+    const int32_t *act;
+    const uint8_t *term, *trunc;
+    float *out;
+    uint32_t A;
+    uint32_t sub_steps;  // steps per staged sub-tile (multiple of 4, <= block size)
+    uint32_t stages;     // ring depth
+    uint32_t tma;        // 1: q / pi are 16-byte aligned at this launch's base
+    float gamma, lambda;
+  };
+  struct Item {
+    float r;
+    uint32_t fl;
+  };
+  struct Nbr {
+    float e, qa, c;
+  };
+  using Aux = NoAux;
+
+  // Dynamic shared memory layout for a chunk of L steps:
+  //   float E[L + 1], Qa[L + 1], C[L + 1]   (index L: first step after the chunk)
+  //   stages x { float q[S * A], pi[S * A] }
+  //   stages x uint64_t mbarrier
+  static __host__ __device__ inline uint32_t scalars_bytes(uint32_t L) {
+    return ((3u * (L + 1u) * 4u) + 15u) & ~15u;
+  }
+  static __host__ __device__ inline uint32_t smem_bytes(uint32_t L, uint32_t S, uint32_t A,
+                                                        uint32_t stages) {
+    return scalars_bytes(L) + stages * 2u * S * A * 4u + stages * 8u;
+  }
+
+  static __device__ __forceinline__ void load(const Args &p, uint32_t i0, int nv, bool vec,
+                                              Item (&it)[4]) {
+    float r[4];
+    load4(p.r, i0, nv, vec, r);
+    uint32_t te = load4_flags(p.term, i0, nv, vec), tr = load4_flags(p.trunc, i0, nv, vec);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) it[k] = Item{r[k], step_flags(te, tr, k)};
+  }
+
+  static __device__ __forceinline__ Nbr nbr_smem(const unsigned char *smem, uint32_t L,
+                                                 uint32_t local) {
+    const float *sE = reinterpret_cast<const float *>(smem);
+    return Nbr{sE[local], sE[(L + 1) + local], sE[2 * (L + 1) + local]};
+  }
+
+  static __device__ __forceinline__ Aff<float> coef(const Args &p, const Item &it, const Nbr &nx,
+                                                    bool row_end, uint32_t n, uint32_t i, Aux &) {
+    bool cont;
+    float nv = successor_value(it.fl, row_end, 0.0f, p.tv, p.boot, n, i, cont);
+    if (cont) return Aff<float>{p.gamma * nx.c, fmaf(p.gamma, fmaf(-nx.c, nx.qa, nx.e), it.r)};
+    return Aff<float>{0.0f, fmaf(p.gamma, nv, it.r)};
+  }
+
+  static __device__ __forceinline__ void emit(const Args &p, uint32_t i0, int nv, bool vec,
+                                              const Item (&)[4], const float (&x)[4],
+                                              const float (&)[4], const Aux (&)[4]) {
+    store4(p.out, i0, nv, vec, x);
+  }
+
+  // E, q_a and c of one step from its staged rows.
+  static __device__ __forceinline__ void reduce_step(const Args &p, const float *qrow,
+                                                     const float *prow, uint32_t step, float &e,
+                                                     float &qa, float &c) {
+    const uint32_t A = p.A;
+    float acc = 0.0f;
+    if ((A & 1u) == 0u) {
+      const float2 *q2 = reinterpret_cast<const float2 *>(qrow);
+      const float2 *p2 = reinterpret_cast<const float2 *>(prow);
+      for (uint32_t a = 0; a < A / 2u; ++a) {
+        float2 qq = q2[a], pp = p2[a];
+        acc = fmaf(pp.x, qq.x, acc);
+        acc = fmaf(pp.y, qq.y, acc);
+      }
+    } else {
+      for (uint32_t a = 0; a < A; ++a) acc = fmaf(prow[a], qrow[a], acc);
+    }
+    const int32_t act = __ldg(p.act + step);
+    const float mu = __ldg(p.mu + step);
+    float qv = 0.0f, pv = 0.0f;
+    if (act >= 0 && uint32_t(act) < A) {
+      qv = qrow[act];
+      pv = prow[act];
+    } else {
+      record_status(kDevStatusInvalidArg);
+    }
+    e = acc;
+    qa = qv;
+    c = p.lambda * fminf(1.0f, pv / mu);
+  }
+
+  // Fill E / Qa / C for the chunk's steps [cbase, cbase + Lc) and the first
+  // step after it (if any).  Ends with a block barrier.
+  static __device__ void prologue(const Args &p, uint32_t cbase, uint32_t L, uint32_t total,
+                                  unsigned char *smem, int tid, int nthreads,
+                                  uint64_t timeout_ns) {
+    float *sE = reinterpret_cast<float *>(smem);
+    float *sQ = sE + (L + 1);
+    float *sC = sQ + (L + 1);
+    const uint32_t A = p.A, S = p.sub_steps, NS = p.stages;
+    float *ring = reinterpret_cast<float *>(smem + scalars_bytes(L));
+    const uint32_t stage_floats = 2u * S * A;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + NS * stage_floats);
+    const uint32_t Lc = min(L, total - cbase);
+    const uint32_t nsub = (Lc + S - 1u) / S;
+    const bool use_tma = p.tma != 0u;
+    auto full = [&](uint32_t j) { return (j + 1u) * S <= Lc; };
+
+    if (use_tma) {
+      if (tid == 0) {
+        for (uint32_t s = 0; s < NS; ++s) mbar_init(&bars[s], 1u);
+        fence_mbar_init();
+      }
+      __syncthreads();
+      if (tid == 0) {
+        for (uint32_t j = 0; j < min(NS, nsub); ++j) {
+          if (!full(j)) break;
+          float *dq = ring + (j % NS) * stage_floats;
+          const uint32_t bytes = S * A * 4u;
+          const size_t off = size_t(cbase + j * S) * A;
+          mbar_arrive_expect_tx(&bars[j % NS], 2u * bytes);
+          bulk_copy_g2s(dq, p.q + off, bytes, &bars[j % NS]);
+          bulk_copy_g2s(dq + S * A, p.pi + off, bytes, &bars[j % NS]);
+        }
+      }
+    }
+
+    // The step after the chunk (its E, q_a, c feed the chunk's last step):
+    // one warp reduces it straight from global memory.
+    if (tid < 32 && cbase + Lc < total) {
+      const uint32_t step = cbase + Lc;
+      const size_t off = size_t(step) * A;
+      float part = 0.0f;
+      for (uint32_t a = tid; a < A; a += 32u) part = fmaf(__ldg(p.pi + off + a), __ldg(p.q + off + a), part);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+      if (tid == 0) {
+        const int32_t act = __ldg(p.act + step);
+        const float mu = __ldg(p.mu + step);
+        float qv = 0.0f, pv = 0.0f;
+        if (act >= 0 && uint32_t(act) < A) {
+          qv = __ldg(p.q + off + act);
+          pv = __ldg(p.pi + off + act);
+        } else {
+          record_status(kDevStatusInvalidArg);
+        }
+        sE[Lc] = part;
+        sQ[Lc] = qv;
+        sC[Lc] = p.lambda * fminf(1.0f, pv / mu);
+      }
+    }
+
+    for (uint32_t j = 0; j < nsub; ++j) {
+      const uint32_t stage = j % NS;
+      float *sq = ring + stage * stage_floats;
+      float *sp = sq + S * A;
+      const uint32_t nst = min(S, Lc - j * S);
+      if (use_tma && full(j)) {
+        mbar_wait_bounded(&bars[stage], (j / NS) & 1u, timeout_ns);
+      } else {
+        const size_t off = size_t(cbase + j * S) * A;
+        for (uint32_t e = tid; e < nst * A; e += nthreads) {
+          sq[e] = __ldg(p.q + off + e);
+          sp[e] = __ldg(p.pi + off + e);
+        }
+        __syncthreads();
+      }
+      if (uint32_t(tid) < nst) {
+        const uint32_t local = j * S + tid;
+        float e, qa, c;
+        reduce_step(p, sq + tid * A, sp + tid * A, cbase + local, e, qa, c);
+        sE[local] = e;
+        sQ[local] = qa;
+        sC[local] = c;
+      }
+      __syncthreads();
+      if (use_tma && tid == 0 && j + NS < nsub && full(j + NS)) {
+        fence_proxy_async_smem();
+        const uint32_t jn = j + NS;
+        const uint32_t bytes = S * A * 4u;
+        const size_t off = size_t(cbase + jn * S) * A;
+        mbar_arrive_expect_tx(&bars[stage], 2u * bytes);
+        bulk_copy_g2s(sq, p.q + off, bytes, &bars[stage]);
+        bulk_copy_g2s(sp, p.pi + off, bytes, &bars[stage]);
+      }
+    }
+  }
+};
+
+}  // namespace rlscan

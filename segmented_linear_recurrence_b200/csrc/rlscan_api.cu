@@ -1,0 +1,671 @@
+// rlscan_api.cu -- host side of librlscan: argument checks, launch plans,
+// look-back workspaces and the extern "C" entry points declared in
+// include/rlscan.h.  Every step of the computation runs in the kernels of
+// scan_kernel.cuh; this file only validates, plans and launches.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "../../include/rlscan.h"
+#include "estimators.cuh"
+#include "retrace.cuh"
+#include "scan_core.cuh"
+#include "scan_kernel.cuh"
+
+using namespace rlscan;
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// options
+// ---------------------------------------------------------------------------
+std::atomic<int64_t> g_timeout_ns{1000000000LL};
+std::atomic<int64_t> g_force_lookback{0};
+std::atomic<int64_t> g_force_block{0};
+std::atomic<int64_t> g_force_scalar{0};
+std::atomic<int64_t> g_check_pointers{1};
+std::atomic<int64_t> g_starve{0};
+
+constexpr int64_t kMaxStepsPerLaunch = int64_t(1) << 30;
+constexpr int64_t kMaxRowSteps = int64_t(1) << 30;
+constexpr int64_t kMaxActions = 2048;
+
+// ---------------------------------------------------------------------------
+// look-back workspaces, one per (device, stream)
+// ---------------------------------------------------------------------------
+struct Workspace {
+  void *ptr = nullptr;
+  size_t bytes = 0;
+};
+std::mutex g_ws_mu;
+std::map<std::pair<int, rlscan_stream_t>, Workspace> g_ws;
+
+rlscan_status get_workspace(rlscan_stream_t stream, size_t need, void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RLSCAN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  Workspace &w = g_ws[{dev, stream}];
+  if (w.bytes >= need) {
+    *out = w.ptr;
+    return RLSCAN_OK;
+  }
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return RLSCAN_ERR_CUDA;
+  if (cs != cudaStreamCaptureStatusNone) return RLSCAN_ERR_CAPTURE;
+  size_t bytes = std::max<size_t>(need, 4096);
+  bytes = (bytes + 4095) & ~size_t(4095);
+  void *p = nullptr;
+  if (w.ptr) {
+    // Stream-ordered: earlier launches on this stream finish with the old block first.
+    if (cudaFreeAsync(w.ptr, stream) != cudaSuccess) return RLSCAN_ERR_CUDA;
+    w.ptr = nullptr;
+    w.bytes = 0;
+  }
+  if (cudaMallocAsync(&p, bytes, stream) != cudaSuccess) {
+    cudaGetLastError();
+    return RLSCAN_ERR_NOMEM;
+  }
+  if (cudaMemsetAsync(p, 0, bytes, stream) != cudaSuccess) {
+    cudaFreeAsync(p, stream);
+    return RLSCAN_ERR_CUDA;
+  }
+  w.ptr = p;
+  w.bytes = bytes;
+  *out = p;
+  return RLSCAN_OK;
+}
+
+// ---------------------------------------------------------------------------
+// argument checks
+// ---------------------------------------------------------------------------
+struct Range {
+  uintptr_t lo, hi;  // [lo, hi)
+};
+
+struct Checker {
+  rlscan_status st = RLSCAN_OK;
+  std::vector<const void *> ptrs;
+  std::vector<Range> in, out;
+
+  void fail(rlscan_status s) {
+    if (st == RLSCAN_OK) st = s;
+  }
+  void need(const void *p) {
+    if (!p) fail(RLSCAN_ERR_INVALID_ARG);
+  }
+  void align(const void *p, uintptr_t a) {
+    if (p && (reinterpret_cast<uintptr_t>(p) % a) != 0) fail(RLSCAN_ERR_INVALID_ARG);
+  }
+  void input(const void *p, size_t bytes, uintptr_t a) {
+    if (!p) return;
+    align(p, a);
+    ptrs.push_back(p);
+    in.push_back({reinterpret_cast<uintptr_t>(p), reinterpret_cast<uintptr_t>(p) + bytes});
+  }
+  void output(void *p, size_t bytes, uintptr_t a) {
+    if (!p) return;
+    align(p, a);
+    ptrs.push_back(p);
+    out.push_back({reinterpret_cast<uintptr_t>(p), reinterpret_cast<uintptr_t>(p) + bytes});
+  }
+  void finite(float x) {
+    if (!std::isfinite(x)) fail(RLSCAN_ERR_INVALID_ARG);
+  }
+  void positive(float x) {
+    if (!(x > 0.0f) || !std::isfinite(x)) fail(RLSCAN_ERR_INVALID_ARG);
+  }
+  static bool overlap(const Range &a, const Range &b) { return a.lo < b.hi && b.lo < a.hi; }
+  void check_overlaps() {
+    for (size_t i = 0; i < out.size(); ++i) {
+      for (size_t j = 0; j < in.size(); ++j)
+        if (overlap(out[i], in[j])) fail(RLSCAN_ERR_OVERLAP);
+      for (size_t j = i + 1; j < out.size(); ++j)
+        if (overlap(out[i], out[j])) fail(RLSCAN_ERR_OVERLAP);
+    }
+  }
+  // Every pointer must be readable by the current device.
+  void check_device_access(rlscan_stream_t stream) {
+    if (st != RLSCAN_OK || g_check_pointers.load() == 0) return;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) {
+      cudaGetLastError();
+      fail(RLSCAN_ERR_CUDA);
+      return;
+    }
+    if (cs != cudaStreamCaptureStatusNone) return;  // checked on the pre-capture call
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+      fail(RLSCAN_ERR_CUDA);
+      return;
+    }
+    for (const void *p : ptrs) {
+      cudaPointerAttributes at;
+      if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        fail(RLSCAN_ERR_INVALID_ARG);
+        return;
+      }
+      bool ok = false;
+      switch (at.type) {
+        case cudaMemoryTypeDevice: ok = at.device == dev; break;
+        case cudaMemoryTypeManaged: ok = true; break;
+        case cudaMemoryTypeHost: ok = at.devicePointer == p; break;
+        default: ok = false; break;
+      }
+      if (!ok) {
+        fail(RLSCAN_ERR_INVALID_ARG);
+        return;
+      }
+    }
+  }
+};
+
+bool dims_ok(int64_t N, int64_t T, int64_t A) {
+  if (N < 0 || T < 0 || A < 1) return false;
+  if (T > 0 && T * A > kMaxRowSteps) return false;
+  if (T > 0 && N > (int64_t(1) << 62) / (T * A)) return false;
+  return true;
+}
+
+bool aligned(const void *p, uintptr_t a) { return p == nullptr || reinterpret_cast<uintptr_t>(p) % a == 0; }
+
+// ---------------------------------------------------------------------------
+// launch plans
+// ---------------------------------------------------------------------------
+struct Plan {
+  int block = 256;
+  uint32_t L = 1024;
+  bool lookback = false;
+  int64_t rows_per_launch = 0;
+  int launches = 0;
+  int64_t blocks = 0;
+  uint32_t max_chunks = 0;
+  size_t ws_bytes = 0;
+  // Retrace staging
+  uint32_t sub_steps = 0, stages = 0;
+  size_t smem = 0;
+};
+
+bool valid_block(int64_t b) { return b == 128 || b == 256 || b == 512 || b == 1024; }
+
+Plan make_plan(rlscan_estimator est, int64_t N, int64_t T, int64_t A) {
+  Plan pl;
+  const int64_t fb = g_force_block.load();
+  if (est == RLSCAN_EST_RETRACE) {
+    pl.block = (fb == 128 || fb == 256) ? int(fb) : 128;
+  } else if (valid_block(fb)) {
+    pl.block = int(fb);
+  } else {
+    pl.block = 0;
+    for (int b : {256, 512, 1024})
+      if ((4 * int64_t(b)) % T == 0) {
+        pl.block = b;
+        break;
+      }
+    if (pl.block == 0) pl.block = 512;
+  }
+  pl.L = 4u * uint32_t(pl.block);
+  pl.lookback = g_force_lookback.load() != 0 || (int64_t(pl.L) % T) != 0;
+  pl.rows_per_launch = std::max<int64_t>(1, kMaxStepsPerLaunch / T);
+  pl.launches = int((N + pl.rows_per_launch - 1) / pl.rows_per_launch);
+  pl.blocks = 0;
+  for (int64_t r0 = 0; r0 < N; r0 += pl.rows_per_launch) {
+    const int64_t rows = std::min(pl.rows_per_launch, N - r0);
+    const uint32_t nch = uint32_t((rows * T + pl.L - 1) / pl.L);
+    pl.blocks += nch;
+    pl.max_chunks = std::max(pl.max_chunks, nch);
+  }
+  pl.ws_bytes = pl.lookback ? sizeof(LookbackHeader) + size_t(pl.max_chunks) * sizeof(LookbackDesc) : 0;
+  if (est == RLSCAN_EST_RETRACE) {
+    // Sub-tile steps and ring depth: the largest staging that keeps at least
+    // three blocks resident per SM (<= ~72 KB of shared memory each).
+    const uint32_t budget = 72u * 1024u;
+    uint32_t S = uint32_t(pl.block);
+    uint32_t NS = 4;
+    while (NS > 2 && RetraceOp::smem_bytes(pl.L, S, uint32_t(A), NS) > budget) --NS;
+    while (S > 4 && RetraceOp::smem_bytes(pl.L, S, uint32_t(A), NS) > budget) S = std::max(4u, (S / 2) & ~3u);
+    pl.sub_steps = S;
+    pl.stages = NS;
+    pl.smem = RetraceOp::smem_bytes(pl.L, S, uint32_t(A), NS);
+  }
+  return pl;
+}
+
+template <class Op, int BLOCK, bool LB>
+cudaError_t launch_kernel(const typename Op::Args &a, const ScanGeom &g, size_t smem,
+                          cudaStream_t s) {
+  auto kern = scan_kernel<Op, BLOCK, LB>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<g.nchunks, BLOCK, smem, s>>>(a, g);
+  return cudaGetLastError();
+}
+
+template <class Op>
+cudaError_t launch_block(const typename Op::Args &a, const ScanGeom &g, int block, bool lb,
+                         size_t smem, cudaStream_t s) {
+  switch (block) {
+    case 128: return lb ? launch_kernel<Op, 128, true>(a, g, smem, s) : launch_kernel<Op, 128, false>(a, g, smem, s);
+    case 256: return lb ? launch_kernel<Op, 256, true>(a, g, smem, s) : launch_kernel<Op, 256, false>(a, g, smem, s);
+    case 512: return lb ? launch_kernel<Op, 512, true>(a, g, smem, s) : launch_kernel<Op, 512, false>(a, g, smem, s);
+    case 1024: return lb ? launch_kernel<Op, 1024, true>(a, g, smem, s) : launch_kernel<Op, 1024, false>(a, g, smem, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <class Op>
+cudaError_t launch_block_retrace(const typename Op::Args &a, const ScanGeom &g, int block, bool lb,
+                                 size_t smem, cudaStream_t s) {
+  switch (block) {
+    case 128: return lb ? launch_kernel<Op, 128, true>(a, g, smem, s) : launch_kernel<Op, 128, false>(a, g, smem, s);
+    case 256: return lb ? launch_kernel<Op, 256, true>(a, g, smem, s) : launch_kernel<Op, 256, false>(a, g, smem, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// Runs every row slice of a call.  `make_args(row0, vec)` returns the
+// estimator's arguments with every pointer advanced to row `row0`; `slice_vec`
+// tells whether that slice's pointers allow vectorised access.
+template <class Op, class MakeArgs, class SliceVec>
+rlscan_status run(const Plan &pl, int64_t N, int64_t T, rlscan_stream_t stream, MakeArgs make_args,
+                  SliceVec slice_vec) {
+  void *ws = nullptr;
+  if (pl.lookback) {
+    rlscan_status s = get_workspace(stream, pl.ws_bytes, &ws);
+    if (s != RLSCAN_OK) return s;
+  }
+  for (int64_t r0 = 0; r0 < N; r0 += pl.rows_per_launch) {
+    const int64_t rows = std::min(pl.rows_per_launch, N - r0);
+    ScanGeom g{};
+    g.total = uint32_t(rows * T);
+    g.T = uint32_t(T);
+    g.nchunks = uint32_t((rows * T + pl.L - 1) / pl.L);
+    const bool vec = g_force_scalar.load() == 0 && slice_vec(r0);
+    g.vec = vec ? 1u : 0u;
+    g.lb.hdr = static_cast<LookbackHeader *>(ws);
+    g.lb.desc = ws ? reinterpret_cast<LookbackDesc *>(static_cast<LookbackHeader *>(ws) + 1) : nullptr;
+    g.lb.timeout_ns = uint64_t(std::max<int64_t>(1000, g_timeout_ns.load()));
+    g.lb.starve = g_starve.load() != 0 ? 1u : 0u;
+    const typename Op::Args a = make_args(r0, vec);
+    cudaError_t e;
+    if constexpr (Op::kPrologue)
+      e = launch_block_retrace<Op>(a, g, pl.block, pl.lookback, pl.smem, stream);
+    else
+      e = launch_block<Op>(a, g, pl.block, pl.lookback, 0, stream);
+    if (e != cudaSuccess) return RLSCAN_ERR_LAUNCH;
+  }
+  return RLSCAN_OK;
+}
+
+template <class T>
+T *adv(T *p, int64_t elems) {
+  return p ? p + elems : nullptr;
+}
+
+}  // namespace
+
+// ===========================================================================
+// extern "C" entry points
+// ===========================================================================
+extern "C" {
+
+rlscan_status rlscan_gae(const float *rewards, const float *values, const float *bootstrap,
+                         const uint8_t *terminated, const uint8_t *truncated,
+                         const float *trunc_value, float *advantages, float *returns, int64_t N,
+                         int64_t T, float gamma, float lambda, rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(rewards), c.need(values), c.need(bootstrap), c.need(advantages);
+  if (truncated) c.need(trunc_value);
+  c.finite(gamma), c.finite(lambda);
+  c.input(rewards, nt * 4, 4), c.input(values, nt * 4, 4), c.input(bootstrap, size_t(N) * 4, 4);
+  c.input(terminated, nt, 1), c.input(truncated, nt, 1);
+  if (truncated) c.input(trunc_value, nt * 4, 4);
+  c.output(advantages, nt * 4, 4), c.output(returns, nt * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  const Plan pl = make_plan(RLSCAN_EST_GAE, N, T, 1);
+  const float *tv = truncated ? trunc_value : nullptr;
+  return run<GaeOp>(
+      pl, N, T, stream,
+      [&](int64_t r0, bool) {
+        const int64_t o = r0 * T;
+        return GaeOp::Args{adv(rewards, o), adv(values, o), adv(bootstrap, r0), adv(tv, o),
+                           adv(terminated, o), adv(truncated, o), adv(advantages, o), adv(returns, o),
+                           gamma, gamma * lambda};
+      },
+      [&](int64_t r0) {
+        const int64_t o = r0 * T;
+        return aligned(adv(rewards, o), 16) && aligned(adv(values, o), 16) &&
+               aligned(adv(advantages, o), 16) && aligned(adv(returns, o), 16) &&
+               aligned(adv(terminated, o), 4) && aligned(adv(truncated, o), 4);
+      });
+}
+
+rlscan_status rlscan_vtrace(const float *log_rhos, const float *rewards, const float *values,
+                            const float *bootstrap, const uint8_t *terminated,
+                            const uint8_t *truncated, const float *trunc_value, float *vs,
+                            float *pg_advantages, int64_t N, int64_t T, float gamma, float lambda,
+                            float rho_bar, float c_bar, rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(log_rhos), c.need(rewards), c.need(values), c.need(bootstrap), c.need(vs);
+  if (truncated) c.need(trunc_value);
+  c.finite(gamma), c.finite(lambda), c.positive(rho_bar), c.positive(c_bar);
+  c.input(log_rhos, nt * 4, 4), c.input(rewards, nt * 4, 4), c.input(values, nt * 4, 4);
+  c.input(bootstrap, size_t(N) * 4, 4), c.input(terminated, nt, 1), c.input(truncated, nt, 1);
+  if (truncated) c.input(trunc_value, nt * 4, 4);
+  c.output(vs, nt * 4, 4), c.output(pg_advantages, nt * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  const Plan pl = make_plan(RLSCAN_EST_VTRACE, N, T, 1);
+  const float *tv = truncated ? trunc_value : nullptr;
+  return run<VtraceOp>(
+      pl, N, T, stream,
+      [&](int64_t r0, bool) {
+        const int64_t o = r0 * T;
+        return VtraceOp::Args{adv(log_rhos, o), adv(rewards, o), adv(values, o), adv(bootstrap, r0),
+                              adv(tv, o), adv(terminated, o), adv(truncated, o), adv(vs, o),
+                              adv(pg_advantages, o), gamma, lambda, rho_bar, c_bar};
+      },
+      [&](int64_t r0) {
+        const int64_t o = r0 * T;
+        return aligned(adv(log_rhos, o), 16) && aligned(adv(rewards, o), 16) &&
+               aligned(adv(values, o), 16) && aligned(adv(vs, o), 16) &&
+               aligned(adv(pg_advantages, o), 16) && aligned(adv(terminated, o), 4) &&
+               aligned(adv(truncated, o), 4);
+      });
+}
+
+rlscan_status rlscan_retrace(const float *q, const float *pi, const float *mu_a,
+                             const int32_t *actions, const float *rewards, const float *bootstrap,
+                             const uint8_t *terminated, const uint8_t *truncated,
+                             const float *trunc_value, float *q_ret, int64_t N, int64_t T,
+                             int64_t A, float gamma, float lambda, rlscan_stream_t stream) {
+  if (A < 1 || A > kMaxActions || !dims_ok(N, T, A)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(q), c.need(pi), c.need(mu_a), c.need(actions), c.need(rewards), c.need(bootstrap);
+  c.need(q_ret);
+  if (truncated) c.need(trunc_value);
+  c.finite(gamma), c.finite(lambda);
+  c.input(q, nt * size_t(A) * 4, 4), c.input(pi, nt * size_t(A) * 4, 4), c.input(mu_a, nt * 4, 4);
+  c.input(actions, nt * 4, 4), c.input(rewards, nt * 4, 4), c.input(bootstrap, size_t(N) * 4, 4);
+  c.input(terminated, nt, 1), c.input(truncated, nt, 1);
+  if (truncated) c.input(trunc_value, nt * 4, 4);
+  c.output(q_ret, nt * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  const Plan pl = make_plan(RLSCAN_EST_RETRACE, N, T, A);
+  const float *tv = truncated ? trunc_value : nullptr;
+  return run<RetraceOp>(
+      pl, N, T, stream,
+      [&](int64_t r0, bool) {
+        const int64_t o = r0 * T;
+        const int64_t oa = o * A;
+        RetraceOp::Args a{};
+        a.q = adv(q, oa), a.pi = adv(pi, oa), a.mu = adv(mu_a, o), a.r = adv(rewards, o);
+        a.boot = adv(bootstrap, r0), a.tv = adv(tv, o), a.act = adv(actions, o);
+        a.term = adv(terminated, o), a.trunc = adv(truncated, o), a.out = adv(q_ret, o);
+        a.A = uint32_t(A), a.sub_steps = pl.sub_steps, a.stages = pl.stages;
+        a.tma = (g_force_scalar.load() == 0 && aligned(a.q, 16) && aligned(a.pi, 16)) ? 1u : 0u;
+        a.gamma = gamma, a.lambda = lambda;
+        return a;
+      },
+      [&](int64_t r0) {
+        const int64_t o = r0 * T;
+        return aligned(adv(rewards, o), 16) && aligned(adv(q_ret, o), 16) &&
+               aligned(adv(terminated, o), 4) && aligned(adv(truncated, o), 4);
+      });
+}
+
+rlscan_status rlscan_td_lambda(const float *rewards, const float *values, const float *bootstrap,
+                               const uint8_t *terminated, const uint8_t *truncated,
+                               const float *trunc_value, float *returns, int64_t N, int64_t T,
+                               float gamma, float lambda, rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(rewards), c.need(values), c.need(bootstrap), c.need(returns);
+  if (truncated) c.need(trunc_value);
+  c.finite(gamma), c.finite(lambda);
+  c.input(rewards, nt * 4, 4), c.input(values, nt * 4, 4), c.input(bootstrap, size_t(N) * 4, 4);
+  c.input(terminated, nt, 1), c.input(truncated, nt, 1);
+  if (truncated) c.input(trunc_value, nt * 4, 4);
+  c.output(returns, nt * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  const Plan pl = make_plan(RLSCAN_EST_TD_LAMBDA, N, T, 1);
+  const float *tv = truncated ? trunc_value : nullptr;
+  return run<TdLambdaOp>(
+      pl, N, T, stream,
+      [&](int64_t r0, bool) {
+        const int64_t o = r0 * T;
+        return TdLambdaOp::Args{adv(rewards, o), adv(values, o), adv(bootstrap, r0), adv(tv, o),
+                                adv(terminated, o), adv(truncated, o), adv(returns, o), gamma,
+                                gamma * lambda, gamma * (1.0f - lambda)};
+      },
+      [&](int64_t r0) {
+        const int64_t o = r0 * T;
+        return aligned(adv(rewards, o), 16) && aligned(adv(values, o), 16) &&
+               aligned(adv(returns, o), 16) && aligned(adv(terminated, o), 4) &&
+               aligned(adv(truncated, o), 4);
+      });
+}
+
+rlscan_status rlscan_discounted_return(const float *rewards, const float *bootstrap,
+                                       const uint8_t *terminated, const uint8_t *truncated,
+                                       const float *trunc_value, float *returns, int64_t N,
+                                       int64_t T, float gamma, rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(rewards), c.need(returns);
+  if (truncated) c.need(trunc_value);
+  c.finite(gamma);
+  c.input(rewards, nt * 4, 4), c.input(bootstrap, size_t(N) * 4, 4);
+  c.input(terminated, nt, 1), c.input(truncated, nt, 1);
+  if (truncated) c.input(trunc_value, nt * 4, 4);
+  c.output(returns, nt * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  const Plan pl = make_plan(RLSCAN_EST_DISCOUNTED_RETURN, N, T, 1);
+  const float *tv = truncated ? trunc_value : nullptr;
+  return run<DiscountedOp>(
+      pl, N, T, stream,
+      [&](int64_t r0, bool) {
+        const int64_t o = r0 * T;
+        return DiscountedOp::Args{adv(rewards, o), adv(bootstrap, r0), adv(tv, o), adv(terminated, o),
+                                  adv(truncated, o), adv(returns, o), gamma};
+      },
+      [&](int64_t r0) {
+        const int64_t o = r0 * T;
+        return aligned(adv(rewards, o), 16) && aligned(adv(returns, o), 16) &&
+               aligned(adv(terminated, o), 4) && aligned(adv(truncated, o), 4);
+      });
+}
+
+rlscan_status rlscan_elig_trace(const float *inputs, const float *init_trace,
+                                const uint8_t *terminated, const uint8_t *truncated,
+                                float *traces, int64_t N, int64_t T, float gamma, float lambda,
+                                rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(inputs), c.need(traces);
+  c.finite(gamma), c.finite(lambda);
+  c.input(inputs, nt * 4, 4), c.input(init_trace, size_t(N) * 4, 4);
+  c.input(terminated, nt, 1), c.input(truncated, nt, 1);
+  c.output(traces, nt * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  const Plan pl = make_plan(RLSCAN_EST_ELIG_TRACE, N, T, 1);
+  return run<EligOp>(
+      pl, N, T, stream,
+      [&](int64_t r0, bool) {
+        const int64_t o = r0 * T;
+        return EligOp::Args{adv(inputs, o), adv(init_trace, r0), adv(terminated, o), adv(truncated, o),
+                            adv(traces, o), gamma * lambda};
+      },
+      [&](int64_t r0) {
+        const int64_t o = r0 * T;
+        return aligned(adv(inputs, o), 16) && aligned(adv(traces, o), 16) &&
+               aligned(adv(terminated, o), 4) && aligned(adv(truncated, o), 4);
+      });
+}
+
+rlscan_status rlscan_episodic_prefix_sum(const int32_t *x, const uint8_t *terminated,
+                                         const uint8_t *truncated, int32_t *out, int64_t N,
+                                         int64_t T, rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(x), c.need(out);
+  c.input(x, nt * 4, 4), c.input(terminated, nt, 1), c.input(truncated, nt, 1);
+  c.output(out, nt * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  const Plan pl = make_plan(RLSCAN_EST_EPISODIC_PREFIX_SUM, N, T, 1);
+  return run<PrefixSumOp>(
+      pl, N, T, stream,
+      [&](int64_t r0, bool) {
+        const int64_t o = r0 * T;
+        return PrefixSumOp::Args{adv(x, o), adv(terminated, o), adv(truncated, o), adv(out, o)};
+      },
+      [&](int64_t r0) {
+        const int64_t o = r0 * T;
+        return aligned(adv(x, o), 16) && aligned(adv(out, o), 16) && aligned(adv(terminated, o), 4) &&
+               aligned(adv(truncated, o), 4);
+      });
+}
+
+rlscan_status rlscan_sync_status(rlscan_stream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) {
+    cudaGetLastError();
+    return RLSCAN_ERR_CUDA;
+  }
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_rlscan_device_status, sizeof(v)) != cudaSuccess) {
+    cudaGetLastError();
+    return RLSCAN_ERR_CUDA;
+  }
+  if (v != 0) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_rlscan_device_status, &zero, sizeof(zero)) != cudaSuccess) {
+      cudaGetLastError();
+      return RLSCAN_ERR_CUDA;
+    }
+  }
+  switch (v) {
+    case kDevStatusOk: return RLSCAN_OK;
+    case kDevStatusInvalidArg: return RLSCAN_ERR_INVALID_ARG;
+    case kDevStatusTimeout: return RLSCAN_ERR_TIMEOUT;
+    default: return RLSCAN_ERR_CUDA;
+  }
+}
+
+const char *rlscan_status_string(rlscan_status s) {
+  switch (s) {
+    case RLSCAN_OK: return "RLSCAN_OK";
+    case RLSCAN_ERR_INVALID_ARG: return "RLSCAN_ERR_INVALID_ARG";
+    case RLSCAN_ERR_OVERLAP: return "RLSCAN_ERR_OVERLAP";
+    case RLSCAN_ERR_LAUNCH: return "RLSCAN_ERR_LAUNCH";
+    case RLSCAN_ERR_TIMEOUT: return "RLSCAN_ERR_TIMEOUT";
+    case RLSCAN_ERR_NOMEM: return "RLSCAN_ERR_NOMEM";
+    case RLSCAN_ERR_CUDA: return "RLSCAN_ERR_CUDA";
+    case RLSCAN_ERR_CAPTURE: return "RLSCAN_ERR_CAPTURE";
+  }
+  return "RLSCAN_ERR_UNKNOWN";
+}
+
+void rlscan_release_workspaces(void) {
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  int cur = 0;
+  const bool have_dev = cudaGetDevice(&cur) == cudaSuccess;
+  for (auto &kv : g_ws) {
+    if (kv.second.ptr) {
+      cudaSetDevice(kv.first.first);
+      cudaFree(kv.second.ptr);
+    }
+  }
+  g_ws.clear();
+  if (have_dev) cudaSetDevice(cur);
+  cudaGetLastError();
+}
+
+int rlscan_abi_version(void) { return RLSCAN_ABI_VERSION; }
+
+rlscan_status rlscan_query_plan(rlscan_estimator est, int64_t N, int64_t T, int64_t A,
+                                rlscan_plan_info *info) {
+  if (!info || int(est) < 0 || int(est) > 6) return RLSCAN_ERR_INVALID_ARG;
+  if (est != RLSCAN_EST_RETRACE) A = 1;
+  if (A < 1 || A > kMaxActions || !dims_ok(N, T, A)) return RLSCAN_ERR_INVALID_ARG;
+  std::memset(info, 0, sizeof(*info));
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  const Plan pl = make_plan(est, N, T, A);
+  info->block_threads = pl.block;
+  info->chunk_steps = int32_t(pl.L);
+  info->lookback = pl.lookback ? 1 : 0;
+  info->launches = pl.launches;
+  info->blocks = pl.blocks;
+  info->workspace_bytes = int64_t(pl.ws_bytes);
+  return RLSCAN_OK;
+}
+
+rlscan_status rlscan_set_option(rlscan_option opt, int64_t v) {
+  switch (opt) {
+    case RLSCAN_OPT_LOOKBACK_TIMEOUT_NS:
+      if (v < 1000) return RLSCAN_ERR_INVALID_ARG;
+      g_timeout_ns = v;
+      return RLSCAN_OK;
+    case RLSCAN_OPT_FORCE_LOOKBACK: g_force_lookback = v ? 1 : 0; return RLSCAN_OK;
+    case RLSCAN_OPT_FORCE_BLOCK:
+      if (v != 0 && !valid_block(v)) return RLSCAN_ERR_INVALID_ARG;
+      g_force_block = v;
+      return RLSCAN_OK;
+    case RLSCAN_OPT_FORCE_SCALAR: g_force_scalar = v ? 1 : 0; return RLSCAN_OK;
+    case RLSCAN_OPT_CHECK_POINTERS: g_check_pointers = v ? 1 : 0; return RLSCAN_OK;
+    case RLSCAN_OPT_TEST_STARVE_LOOKBACK: g_starve = v ? 1 : 0; return RLSCAN_OK;
+  }
+  return RLSCAN_ERR_INVALID_ARG;
+}
+
+int64_t rlscan_get_option(rlscan_option opt) {
+  switch (opt) {
+    case RLSCAN_OPT_LOOKBACK_TIMEOUT_NS: return g_timeout_ns.load();
+    case RLSCAN_OPT_FORCE_LOOKBACK: return g_force_lookback.load();
+    case RLSCAN_OPT_FORCE_BLOCK: return g_force_block.load();
+    case RLSCAN_OPT_FORCE_SCALAR: return g_force_scalar.load();
+    case RLSCAN_OPT_CHECK_POINTERS: return g_check_pointers.load();
+    case RLSCAN_OPT_TEST_STARVE_LOOKBACK: return g_starve.load();
+  }
+  return -1;
+}
+
+}  // extern "C"

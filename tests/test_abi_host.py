@@ -1,0 +1,171 @@
+"""Host-only checks of the C ABI boundary (no GPU needed).
+
+The library must load, export every entry point include/rlscan.h declares,
+and reject invalid arguments synchronously -- before any CUDA call -- with the
+documented status codes.  Fake (never dereferenced) addresses are used for
+the pointers: argument checks run before anything touches them.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import segmented_linear_recurrence_b200 as slr
+from segmented_linear_recurrence_b200 import build as slr_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rlscan.h")
+
+OK, INVALID, OVERLAP = 0, 1, 2
+
+
+@pytest.fixture(scope="module")
+def L():
+    slr_build.build()
+    return slr.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(rlscan_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_seven_estimators():
+    names = declared_functions()
+    for est in ("gae", "vtrace", "retrace", "td_lambda", "discounted_return", "elig_trace",
+                "episodic_prefix_sum"):
+        assert f"rlscan_{est}" in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", slr.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (rlscan_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(L, n)
+
+
+def test_abi_version_and_status_strings(L):
+    assert slr.rlscan_abi_version() == 1
+    for code, name in slr.STATUS.items():
+        assert slr.rlscan_status_string(code) == name
+    assert slr.rlscan_status_string(99) == "RLSCAN_ERR_UNKNOWN"
+
+
+def P(addr):
+    return ctypes.c_void_p(addr)
+
+
+BASE = 0x7F0000000000  # a fake, 256-byte aligned address range; never dereferenced
+
+
+def gae(L, N=4, T=8, r=BASE, v=BASE + 0x10000, b=BASE + 0x20000, te=BASE + 0x30000, tr=None,
+        tv=None, adv=BASE + 0x40000, ret=BASE + 0x50000, g=0.99, lam=0.95):
+    return L.rlscan_gae(P(r), P(v), P(b), P(te) if te else None, P(tr) if tr else None,
+                        P(tv) if tv else None, P(adv) if adv else None, P(ret) if ret else None,
+                        N, T, g, lam, None)
+
+
+def test_empty_problem_is_a_noop(L):
+    assert gae(L, N=0, T=8, r=0, v=0, b=0, te=0, adv=0, ret=0) == OK
+    assert gae(L, N=5, T=0, r=0, v=0, b=0, te=0, adv=0, ret=0) == OK
+    assert L.rlscan_episodic_prefix_sum(None, None, None, None, 0, 0, None) == OK
+
+
+def test_negative_sizes_rejected(L):
+    assert gae(L, N=-1) == INVALID
+    assert gae(L, T=-3) == INVALID
+
+
+def test_null_mandatory_pointers_rejected(L):
+    assert gae(L, r=0) == INVALID
+    assert gae(L, v=0) == INVALID
+    assert gae(L, b=0) == INVALID
+    assert gae(L, adv=0) == INVALID
+    # truncated given without trunc_value
+    assert gae(L, tr=BASE + 0x60000, tv=0) == INVALID
+
+
+def test_misaligned_float_pointer_rejected(L):
+    assert gae(L, r=BASE + 2) == INVALID
+
+
+def test_non_finite_scalars_rejected(L):
+    assert gae(L, g=float("nan")) == INVALID
+    assert gae(L, lam=float("inf")) == INVALID
+    vp = [P(BASE + i * 0x10000) for i in range(9)]
+    st = L.rlscan_vtrace(vp[0], vp[1], vp[2], vp[3], vp[4], None, None, vp[5], vp[6], 4, 8, 0.99,
+                         1.0, 0.0, 1.0, None)
+    assert st == INVALID  # rho_bar must be > 0
+
+
+def test_overlapping_outputs_rejected(L):
+    # output overlapping an input (in-place) and two overlapping outputs
+    assert gae(L, adv=BASE) == OVERLAP
+    assert gae(L, ret=BASE + 0x40000 + 16) == OVERLAP
+    # adjacent, non-overlapping buffers are fine up to the device check
+    N, T = 4, 8
+    st = gae(L, N=N, T=T, adv=BASE + 0x40000, ret=BASE + 0x40000 + N * T * 4)
+    assert st != OVERLAP
+
+
+def test_retrace_action_dim_limits(L):
+    vp = [P(BASE + i * 0x100000) for i in range(10)]
+    args = vp[:9] + [vp[9]]
+    assert L.rlscan_retrace(*args, 4, 8, 0, 0.99, 0.95, None) == INVALID
+    assert L.rlscan_retrace(*args, 4, 8, 4096, 0.99, 0.95, None) == INVALID
+    assert L.rlscan_retrace(*args, 2, 1 << 20, 1 << 11, 0.99, 0.95, None) == INVALID  # T*A > 2^30
+
+
+def test_valid_call_without_gpu_reports_cuda_error(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert gae(L) not in (OK, INVALID, OVERLAP)
+
+
+def test_query_plan(L):
+    p = slr.rlscan_query_plan("gae", 4096, 512)
+    assert p["lookback"] == 0 and p["chunk_steps"] % 512 == 0 and p["launches"] == 1
+    assert p["blocks"] == 4096 * 512 // p["chunk_steps"]
+    p = slr.rlscan_query_plan("vtrace", 256, 16384)
+    assert p["lookback"] == 1 and p["workspace_bytes"] >= 16 * p["blocks"]
+    p = slr.rlscan_query_plan("retrace", 2048, 512, 18)
+    assert p["lookback"] == 0 and p["block_threads"] in (128, 256)
+    p = slr.rlscan_query_plan("episodic_prefix_sum", 3, 33)
+    assert p["lookback"] == 1
+    # more steps than one launch takes are split by rows
+    p = slr.rlscan_query_plan("discounted_return", 1 << 12, 1 << 19)
+    assert p["launches"] == 2
+    assert slr.rlscan_query_plan("gae", 0, 5)["blocks"] == 0
+
+
+def test_options_roundtrip(L):
+    for name, default in (("lookback_timeout_ns", 10 ** 9), ("force_lookback", 0),
+                          ("force_block", 0), ("force_scalar", 0), ("check_pointers", 1),
+                          ("test_starve_lookback", 0)):
+        assert slr.rlscan_get_option(name) == default
+    slr.rlscan_set_option("force_block", 512)
+    assert slr.rlscan_query_plan("gae", 64, 32)["block_threads"] == 512
+    slr.rlscan_set_option("force_block", 0)
+    with pytest.raises(slr.RlscanError):
+        slr.rlscan_set_option("force_block", 100)
+    with pytest.raises(slr.RlscanError):
+        slr.rlscan_set_option("lookback_timeout_ns", 10)
+    slr.rlscan_set_option("force_lookback", 1)
+    assert slr.rlscan_query_plan("gae", 64, 32)["lookback"] == 1
+    slr.rlscan_set_option("force_lookback", 0)
+
+
+def test_binding_raises_without_gpu():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    r = torch.zeros(2, 4)
+    with pytest.raises(RuntimeError):
+        slr.rlscan_discounted_return(r, None, torch.zeros(2, 4, dtype=torch.uint8))

@@ -1,0 +1,113 @@
+"""GPU checks of the launch plans and of the bounded look-back wait.
+
+The same inputs go through every block size, the look-back path forced on
+where whole rows fit a block, and the scalar (unvectorised) path; each must
+match the oracle.  The fault test makes one block withhold its carry (a flag
+that nothing sets): its dependants must give up after the configured wait,
+report RLSCAN_ERR_TIMEOUT through rlscan_sync_status, and leave the context
+usable for the next call.
+"""
+import numpy as np
+import pytest
+import torch
+
+import segmented_linear_recurrence_b200 as slr
+from segmented_linear_recurrence_b200 import synthetic
+from segmented_linear_recurrence_b200 import build as slr_build
+
+from .util import check, f32_scalars, gpu_run
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    slr_build.build()
+
+
+@pytest.fixture
+def options():
+    yield slr.rlscan_set_option
+    for name, default in (("force_lookback", 0), ("force_block", 0), ("force_scalar", 0),
+                          ("test_starve_lookback", 0), ("lookback_timeout_ns", 10 ** 9)):
+        slr.rlscan_set_option(name, default)
+
+
+PLAN_CASES = [(4096 // 8, 128), (64, 2048), (5, 5000), (40, 96)]
+
+
+@pytest.mark.parametrize("est", synthetic.ESTIMATORS)
+@pytest.mark.parametrize("block", [128, 256, 512, 1024])
+@pytest.mark.parametrize("lookback", [0, 1])
+def test_every_plan_matches_oracle(est, block, lookback, options):
+    if est == "retrace" and block > 256:
+        pytest.skip("Retrace stages its action rows with 128- or 256-thread blocks")
+    options("force_block", block)
+    options("force_lookback", lookback)
+    for N, T in PLAN_CASES:
+        d = synthetic.make_inputs(est, N, T, seed=900 + N + T, p_term=0.01, p_trunc=0.01, A=6,
+                                  with_init=True)
+        plan = slr.rlscan_query_plan(est, N, T, 6)
+        assert plan["block_threads"] == (block if est != "retrace" or block <= 256 else 128)
+        if lookback:
+            assert plan["lookback"] == 1
+        check(est, d, synthetic.SCALARS[est], what=f"block={block} lookback={lookback} N={N} T={T}")
+
+
+@pytest.mark.parametrize("est", synthetic.ESTIMATORS)
+def test_scalar_path_matches_vector_path(est, options):
+    d = synthetic.make_inputs(est, 48, 1536, seed=71, p_term=0.01, p_trunc=0.01, A=6,
+                              with_init=True)
+    s = f32_scalars(est, synthetic.SCALARS[est])
+    vec = gpu_run(est, d, **s)
+    options("force_scalar", 1)
+    sca = gpu_run(est, d, **s)
+    for a, b in zip(vec, sca):
+        if a is not None:
+            np.testing.assert_array_equal(a, b)
+
+
+def test_lookback_survives_many_calls_on_one_stream(options):
+    # the per-stream workspace is reused: tickets wrap and the epoch advances
+    d = synthetic.make_inputs("td_lambda", 8, 30_000, seed=72, p_term=0.0005)
+    s = f32_scalars("td_lambda", synthetic.SCALARS["td_lambda"])
+    first = gpu_run("td_lambda", d, **s)
+    for _ in range(20):
+        np.testing.assert_array_equal(first[0], gpu_run("td_lambda", d, **s)[0])
+    d2 = synthetic.make_inputs("td_lambda", 3, 70_001, seed=73, p_term=0.0005)
+    check("td_lambda", d2, synthetic.SCALARS["td_lambda"], what="grown workspace")
+    assert slr.rlscan_sync_status() == 0
+
+
+def test_lookback_on_two_streams(options):
+    d = synthetic.make_inputs("gae", 4, 50_000, seed=74, p_term=0.0005, p_trunc=0.0005)
+    s = f32_scalars("gae", synthetic.SCALARS["gae"])
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    with torch.cuda.stream(s1):
+        a = gpu_run("gae", d, stream=s1, **s)
+    with torch.cuda.stream(s2):
+        b = gpu_run("gae", d, stream=s2, **s)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_withheld_carry_times_out_and_reports(options):
+    # Two rows of 40_000 steps: 10 chunks per row with 1024-step chunks.  The
+    # block holding the first ticket (the last chunk of the last row) never
+    # publishes; the chunk before it waits 20 ms, gives up and reports.
+    options("lookback_timeout_ns", 20_000_000)
+    options("force_block", 256)
+    options("test_starve_lookback", 1)
+    d = synthetic.make_inputs("discounted_return", 2, 40_000, seed=75, p_term=0.0)
+    d["terminated"][:] = 0
+    s = f32_scalars("discounted_return", synthetic.SCALARS["discounted_return"])
+    assert slr.rlscan_sync_status() == 0
+    gpu_run("discounted_return", d, **s)
+    assert slr.rlscan_sync_status() == 4  # RLSCAN_ERR_TIMEOUT
+    # the context stays usable and the next call is correct
+    options("test_starve_lookback", 0)
+    check("discounted_return", d, synthetic.SCALARS["discounted_return"], what="after timeout")
+    assert slr.rlscan_sync_status() == 0

@@ -106,6 +106,30 @@ def load_traffic(kernel_key: str):
 
 
 # ---------------------------------------------------------------------------
+# multi-rank host logic (weak scaling over independent env shards)
+# ---------------------------------------------------------------------------
+def shard_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own rollout shard: same shapes, different data."""
+    return base_seed + 7919 * rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank device-timed duration over all ranks (no-op alone)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(world: int, units_per_rank: int, max_ms: float) -> float:
+    """Whole-job throughput: units all ranks processed / the slowest rank's time."""
+    return world * units_per_rank / (max_ms / 1000.0)
+
+
+# ---------------------------------------------------------------------------
 # clocks
 # ---------------------------------------------------------------------------
 class ClockSampler:
@@ -176,7 +200,7 @@ def workload_calls(workload: str, rank: int):
     calls = []
     for est in w["estimators"]:
         for T in w["Ts"]:
-            seed = synthetic.seed_for(workload, est, T) + 7919 * rank
+            seed = shard_seed(synthetic.seed_for(workload, est, T), rank)
             d = synthetic.make_inputs(est, w["N"], T, seed=seed, p_term=w["p_term"],
                                       p_trunc=w["p_trunc"], A=w.get("A", 18))
             calls.append((est, T, d))
@@ -226,68 +250,97 @@ def run_gpu(args, rank, world, local_rank):
         for c in calls:
             c.launch()
 
-    # warm-up: one eager step (allocates any look-back workspace), then graphs
+    # warm-up: one eager step on the capture stream (so its workspace exists
+    # before capture), then graph replays
+    cap_stream = torch.cuda.Stream(device)
+    ws = 0
+    for est, T, d in host_calls:
+        A = d["q"].shape[2] if est == "retrace" else 1
+        N = d["q"].shape[0] if est == "retrace" else d[ARG_ORDER[est][0]].shape[0]
+        ws = max(ws, slr.rlscan_query_plan(est, N, T, A)["workspace_bytes"])
+    slr.rlscan_reserve_workspace(ws, cap_stream)
     warm_done = 0
-    eager_step()
+    with torch.cuda.stream(cap_stream):
+        eager_step()
     warm_done += 1
     torch.cuda.synchronize()
     if slr.rlscan_sync_status() != 0:
         raise RuntimeError("device status error during warm-up")
 
-    P = max(1, min(args.steps, 8))
-    graphs, events = [], []
-    for _ in range(P):
+    def capture(marks):
+        """A graph of one step; `marks` = indices of calls preceded by a timing event
+        (plus one event after the last call).  Returns (graph, events)."""
         g = torch.cuda.CUDAGraph()
-        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
-        with torch.cuda.graph(g, stream=torch.cuda.Stream(device)):
+        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(marks) + 1)]
+        with torch.cuda.graph(g, stream=cap_stream):
             cur = torch.cuda.current_stream()
-            evs[0].record(cur)
+            e = 0
             for j, c in enumerate(calls):
+                if e < len(marks) and marks[e] == j:
+                    evs[e].record(cur)
+                    e += 1
                 c.launch()
-                evs[j + 1].record(cur)
-        graphs.append(g)
-        events.append(evs)
+            evs[-1].record(cur)
+        return g, evs
+
+    # plain step graph (timed: value), per-estimator-group events (timed:
+    # roofline), per-launch events (diagnostic per-T table)
+    g_plain, _ = capture([])
+    groups = []
+    for j, c in enumerate(calls):
+        if j == 0 or calls[j - 1].est != c.est:
+            groups.append(j)
+    g_group, ev_group = capture(groups)
+    g_each, ev_each = capture(list(range(len(calls))))
     while warm_done < max(args.warmup, 1):
-        graphs[warm_done % P].replay()
+        g_plain.replay()
         warm_done += 1
+    g_group.replay()
+    g_each.replay()
     torch.cuda.synchronize()
 
     gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
     sampler = ClockSampler(gpu_uuid)
     time.sleep(0.3)  # let the sampler start before the timed region
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for k in range(args.steps):
-        graphs[k % P].replay()
-    t1.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+
+    def timed(graph, per_step_events=None):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        acc = None if per_step_events is None else np.zeros(len(per_step_events) - 1)
+        t0.record(stream)
+        for k in range(args.steps):
+            graph.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        if per_step_events is not None:  # the last replay's intervals
+            acc = np.array([per_step_events[i].elapsed_time(per_step_events[i + 1])
+                            for i in range(len(per_step_events) - 1)])
+        return t0.elapsed_time(t1), acc
+
+    elapsed_ms, _ = timed(g_plain)
+    group_ms_total, group_last = timed(g_group, ev_group)
     clocks = sampler.stop()
-    elapsed_ms = t0.elapsed_time(t1)
+    _, each_last = timed(g_each, ev_each)
     status = slr.rlscan_sync_status()
-
-    # per-launch durations (last replay of each graph in the timed region)
-    per_call_ms = np.zeros(len(calls))
-    for evs in events:
-        for j in range(len(calls)):
-            per_call_ms[j] += evs[j].elapsed_time(evs[j + 1])
-    per_call_ms /= P
-
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    # per-group time averaged over the whole group-timed region: scale the last
+    # replay's split by the region's total
+    group_ms = group_last * (group_ms_total / args.steps) / max(group_last.sum(), 1e-9)
+    per_group = {calls[j].est: float(group_ms[i]) for i, j in enumerate(groups)}
+    per_call_ms = each_last
+    del g_plain, g_group, g_each
+    max_ms = max_over_ranks(elapsed_ms, device)
 
     # e2e: the same step through the public API from pinned host buffers
     e2e = run_e2e(args, host_calls, device, world)
 
     return dict(calls=calls, steps_per_step=steps_per_step, launches_per_step=launches_per_step,
-                elapsed_ms=max_ms, per_call_ms=per_call_ms, clocks=clocks, e2e=e2e,
+                elapsed_ms=max_ms, per_call_ms=per_call_ms, per_group=per_group,
+                group_ms_per_step=group_ms_total / args.steps, clocks=clocks, e2e=e2e,
                 warmup=warm_done, status=status)
 
 
@@ -325,10 +378,8 @@ def run_e2e(args, host_calls, device, world):
         step()
     b.record()
     torch.cuda.synchronize()
-    ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-    return dict(ms_per_step=float(ms.item()) / n, steps=n, h2d=h2d, d2h=d2h)
+    ms = max_over_ranks(a.elapsed_time(b), device)
+    return dict(ms_per_step=ms / n, steps=n, h2d=h2d, d2h=d2h)
 
 
 # ---------------------------------------------------------------------------
@@ -424,21 +475,24 @@ def main():
 
     calls = res["calls"]
     ms_step = res["elapsed_ms"] / args.steps
-    value = world * res["steps_per_step"] / (ms_step / 1000.0)
+    value = aggregate_rate(world, res["steps_per_step"], ms_step)
     peak, peak_kind = measured_peak()
 
-    # per-estimator breakdown and the dominant kernel
+    # per-estimator breakdown (group events, timed over K steps) and the
+    # dominant kernel; per-T launch times from the per-launch-event graph
     per_est = {}
     for c, ms in zip(calls, res["per_call_ms"]):
-        e = per_est.setdefault(c.est, {"ms": 0.0, "bytes": 0, "launches": 0, "by_T": {}})
-        e["ms"] += ms
+        e = per_est.setdefault(c.est, {"bytes": 0, "steps": 0, "launches": 0, "by_T": {}})
         e["bytes"] += c.bytes
+        e["steps"] += c.steps
         e["launches"] += 1
         gbs = c.bytes / (ms / 1000.0) / 1e9
         e["by_T"][str(c.T)] = {"us": round(ms * 1000.0, 2),
                                "gsteps_s": round(c.steps / (ms / 1000.0) / 1e9, 2),
                                "gbs": round(gbs, 1), "frac_of_measured": round(gbs / peak, 3),
                                "frac_of_8TBs": round(gbs / SPEC_HBM_GBS, 3)}
+    for est, e in per_est.items():
+        e["ms"] = res["per_group"][est]
     dom = max(per_est, key=lambda k: per_est[k]["ms"])
     de = per_est[dom]
     achieved = de["bytes"] / (de["ms"] / 1000.0) / 1e9
@@ -449,10 +503,12 @@ def main():
                 "kernel": dom_kernel, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
                 "algorithmic_bytes_per_launch": int(de["bytes"] / de["launches"]),
                 "avg_launch_us": round(1000.0 * de["ms"] / de["launches"], 2),
-                "frac_of_8TBs_spec": round(achieved / SPEC_HBM_GBS, 4)}
+                "frac_of_8TBs_spec": round(achieved / SPEC_HBM_GBS, 4),
+                "timing": "CUDA events around each estimator's launches inside the step graph, "
+                          "averaged over the K timed steps"}
 
     e2e = res["e2e"]
-    e2e_value = world * res["steps_per_step"] / (e2e["ms_per_step"] / 1000.0)
+    e2e_value = aggregate_rate(world, res["steps_per_step"], e2e["ms_per_step"])
 
     w = synthetic.WORKLOADS[args.workload]
     line = {
@@ -465,7 +521,7 @@ def main():
                    "l2": "inputs > L2: every call reads its own buffers; "
                          f"{sum(sum(x.numel() * x.element_size() for x in c.inputs if x is not None) for c in calls) / 1e9:.2f}"
                          " GB of distinct inputs per step",
-                   "timing": "CUDA-graph replay of each step; timing-event nodes between launches",
+                   "timing": "K replays of a CUDA graph holding one step's launches, CUDA events around the K",
                    "parallelism": f"dp{world} (independent env shards, no collective)"},
         "roofline": roofline,
         "gpu_launches": int(res["launches_per_step"] * args.steps),
@@ -473,9 +529,12 @@ def main():
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(e2e["h2d"]),
                 "d2h_bytes_per_step": int(e2e["d2h"]), "ms_per_step": e2e["ms_per_step"],
                 "steps": e2e["steps"], "path": "public Python API on pinned host tensors"},
-        "per_estimator": {k: {"gbs": round(v["bytes"] / (v["ms"] / 1000.0) / 1e9, 1),
+        "per_estimator": {k: {"gsteps_s": round(v["steps"] / (v["ms"] / 1000.0) / 1e9, 2),
+                              "gbs": round(v["bytes"] / (v["ms"] / 1000.0) / 1e9, 1),
                               "frac_of_measured": round(v["bytes"] / (v["ms"] / 1000.0) / 1e9 / peak, 4),
-                              "by_T": v["by_T"]} for k, v in per_est.items()},
+                              "ms_per_step": round(v["ms"], 4),
+                              "by_T_event_per_launch": v["by_T"]} for k, v in per_est.items()},
+        "ms_per_step_with_group_events": res["group_ms_per_step"],
         "device_status": res["status"],
     }
     if rank == 0 and world == 1 and args.cpu_seconds > 0:

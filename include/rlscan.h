@@ -25,9 +25,10 @@
  *   nonzero meaning true (the byte layout of torch.bool).
  * Pointers.  Every pointer is a device-accessible address (device, managed or
  *   mapped pinned host memory) on the current CUDA device.  Float and int32
- *   arrays must be 4-byte aligned; 16-byte alignment of every array (and
- *   4-byte alignment of flag arrays) selects the vectorised path, anything
- *   else the scalar path with the same results.  The caller owns every buffer.
+ *   arrays must be 4-byte aligned.  32-byte alignment of every per-step array
+ *   (8-byte for flag arrays; Retrace: 16 and 4) selects the vectorised path,
+ *   anything else the scalar path with the same results.  The caller owns
+ *   every buffer.
  *   Outputs must not overlap any input or each other (in-place use is refused:
  *   the kernels read neighbouring steps).
  * Episode boundaries (same page, Methodologie 3 "Expliciete Boundary
@@ -46,12 +47,13 @@
  * Scalars.  gamma, lambda, rho_bar, c_bar must be finite; rho_bar, c_bar > 0.
  * Streams.  Every call is asynchronous on `stream` (NULL = legacy default
  *   stream).  Calls on different streams may run concurrently.
- * Scratch.  Long rows (more steps than one thread block holds) are split
- *   across thread blocks that hand their carries to one another through a
- *   small per-(device, stream) workspace the library allocates on the first
- *   such call and keeps until rlscan_release_workspaces().  Allocation is not
- *   allowed while `stream` is being captured into a CUDA graph: make one call
- *   of the same or larger size on that stream before capturing.
+ * Scratch.  Thread blocks draw chunks of work from a ticket counter, and long
+ *   rows (more steps than one chunk) are split across chunks that hand their
+ *   carries to one another; both live in a small per-(device, stream)
+ *   workspace the library allocates on the first call on that stream and
+ *   keeps until rlscan_release_workspaces().  Allocation is not allowed while
+ *   `stream` is being captured into a CUDA graph: make one call of the same or
+ *   larger size on that stream before capturing.
  * Errors.  Invalid arguments are reported synchronously and launch nothing.
  *   Conditions only the device can see (a carry hand-off that timed out, an
  *   action index outside [0, A)) are recorded in a per-device status word
@@ -196,6 +198,12 @@ const char *rlscan_status_string(rlscan_status status);
  * caller must ensure no rlscan work is in flight. */
 void rlscan_release_workspaces(void);
 
+/* Make sure the workspace of (current device, `stream`) holds at least
+ * `bytes` (as reported by rlscan_query_plan's workspace_bytes), allocating it
+ * now.  Call before capturing work on `stream` into a CUDA graph.
+ * RLSCAN_ERR_CAPTURE if the stream is capturing and the workspace is too small. */
+rlscan_status rlscan_reserve_workspace(int64_t bytes, rlscan_stream_t stream);
+
 /* ABI version this library was built with (RLSCAN_ABI_VERSION). */
 int rlscan_abi_version(void);
 
@@ -215,8 +223,9 @@ typedef struct rlscan_plan_info {
   int32_t chunk_steps;      /* steps one thread block scans */
   int32_t lookback;         /* 1: blocks chain their carries through the workspace */
   int32_t launches;         /* kernel launches the call makes (row slices) */
-  int64_t blocks;           /* thread blocks over all launches */
-  int64_t workspace_bytes;  /* workspace the call needs on its stream (0 without lookback) */
+  int64_t chunks;           /* chunks of chunk_steps steps over all launches; persistent
+                               blocks draw them from a ticket counter */
+  int64_t workspace_bytes;  /* workspace the call needs on its stream */
 } rlscan_plan_info;
 
 rlscan_status rlscan_query_plan(rlscan_estimator estimator, int64_t N, int64_t T, int64_t A,
@@ -226,7 +235,8 @@ rlscan_status rlscan_query_plan(rlscan_estimator estimator, int64_t N, int64_t T
 typedef enum rlscan_option {
   RLSCAN_OPT_LOOKBACK_TIMEOUT_NS = 1, /* carry wait limit per block, default 1e9 (1 s) */
   RLSCAN_OPT_FORCE_LOOKBACK = 2,      /* 1: chain carries even where blocks hold whole rows */
-  RLSCAN_OPT_FORCE_BLOCK = 3,         /* 0: auto; else threads per block (128, 256, 512, 1024) */
+  RLSCAN_OPT_FORCE_BLOCK = 3,         /* 0: auto; else threads per block (128, 256, 512;
+                                         Retrace takes 128 or 256 and ignores other values) */
   RLSCAN_OPT_FORCE_SCALAR = 4,        /* 1: take the scalar (unvectorised) load path */
   RLSCAN_OPT_CHECK_POINTERS = 5,      /* default 1: reject host memory the device cannot read */
   RLSCAN_OPT_TEST_STARVE_LOOKBACK = 6 /* test only, 1: the first block never publishes its

@@ -24,6 +24,7 @@ __all__ = [
     "rlscan_discounted_return", "rlscan_elig_trace", "rlscan_episodic_prefix_sum",
     "rlscan_sync_status", "rlscan_status_string", "rlscan_release_workspaces",
     "rlscan_abi_version", "rlscan_query_plan", "rlscan_set_option", "rlscan_get_option",
+    "rlscan_reserve_workspace",
     "STATUS", "OPTIONS", "ESTIMATOR_IDS", "LIB_PATH",
 ]
 
@@ -47,7 +48,7 @@ class RlscanError(RuntimeError):
 class PlanInfo(ctypes.Structure):
     _fields_ = [("block_threads", ctypes.c_int32), ("chunk_steps", ctypes.c_int32),
                 ("lookback", ctypes.c_int32), ("launches", ctypes.c_int32),
-                ("blocks", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
+                ("chunks", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
 
 
 _lib = None
@@ -62,6 +63,7 @@ _SIGNATURES = {
     "rlscan_episodic_prefix_sum": [_VP] * 4 + [_I64, _I64, _VP],
     "rlscan_sync_status": [_VP],
     "rlscan_release_workspaces": [],
+    "rlscan_reserve_workspace": [_I64, _VP],
     "rlscan_abi_version": [],
     "rlscan_query_plan": [_I, _I64, _I64, _I64, ctypes.POINTER(PlanInfo)],
     "rlscan_set_option": [_I, _I64],
@@ -322,6 +324,14 @@ def rlscan_status_string(status: int) -> str:
 
 def rlscan_release_workspaces():
     lib().rlscan_release_workspaces()
+
+
+def rlscan_reserve_workspace(nbytes: int, stream=None):
+    """Allocate the (device, stream) workspace now, e.g. before graph capture."""
+    s = torch.cuda.current_stream() if stream is None else stream
+    st = lib().rlscan_reserve_workspace(int(nbytes), ctypes.c_void_p(s.cuda_stream))
+    if st != 0:
+        raise RlscanError("rlscan_reserve_workspace", st)
 
 
 def rlscan_abi_version() -> int:

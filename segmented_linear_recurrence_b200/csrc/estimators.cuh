@@ -6,23 +6,26 @@
 // recurrence coefficients in registers; they are never written to HBM.  Each
 // struct below is one estimator: which arrays it streams, how a step's
 // (a_t, b_t) follow from them and from the neighbouring step, and which
-// outputs it derives from the solved x_t.  The formulas are the estimators'
-// original papers' (listed per struct); the boundary rules are Methodologie 3
+// outputs derive from the solved x_t.  The formulas are the estimators'
+// original papers' (named per struct); the boundary rules are Methodologie 3
 // of the same page: termination -> successor value 0, truncation ->
 // trunc_value, window end -> bootstrap, counted once in the local term.
 //
-// Interface used by scan_kernel.cuh (all members static __device__):
-//   V                value type of the scan (float, or uint32_t for integers)
-//   kBackward        true: x_t = b_t + a_t x_{t+1};  false: x_t = b_t + a_t x_{t-1}
-//   kNeedsNbr        whether coef() reads the neighbouring step (t+1 / t-1)
-//   kPrologue        whether per-step inputs are first reduced into shared memory
-//   Args, Item, Nbr, Aux
-//   load(args, i0, nvalid, vec, item[4])      4 consecutive steps starting at i0
-//   nbr_of(item) / nbr_load(args, i)          what a step gives its neighbour
-//   coef(args, item, nbr, row_edge, n, i, aux) -> Aff<V>
-//   emit(args, i0, nvalid, vec, item, x, x_dep, aux)
-//     x[k] is the solved value at step i0+k and x_dep[k] the value it was
-//     derived from (x_{t+1} backward, x_{t-1} forward).
+// A thread owns a tile of K = 8 consecutive steps: one 256-bit load per fp32
+// array, one 64-bit load per flag array.  Interface used by scan_kernel.cuh
+// (all members static __device__):
+//   V, kBackward, Args, Raw
+//   load(args, tile, lane, total, raw)   issues every load whose address is
+//        known from the tile's position alone: the per-step arrays, the halo
+//        step across the lane edge (lane 31 backward / lane 0 forward) and the
+//        per-row value (bootstrap / initial trace) of the tile's row edge
+//   nbr_of(raw) / halo_of(raw)           the step a neighbouring lane needs
+//   coef(args, tile, fd, raw, nbr, c)    fills the 8 coefficients; the only
+//        data-dependent loads (trunc_value where truncated) are issued here;
+//        may keep per-step state in `raw` for emit()
+//   emit(args, tile, raw, c, x, xdep)    writes the outputs
+// x[k] is the solved value at step k, xdep[k] the one it was derived from
+// (x_{t+1} backward, x_{t-1} forward).
 #pragma once
 
 #include <cstdint>
@@ -32,96 +35,116 @@
 
 namespace rlscan {
 
+constexpr int kTile = 8;  // consecutive steps per thread
+
+// Geometry of one thread's tile.
+struct Tile {
+  uint32_t i0;     // first step (flat, launch-local)
+  int nvalid;      // steps of the tile inside the launch (0..8)
+  uint32_t valid;  // bit k: step k exists
+  uint32_t n0, t0; // row and time of step i0
+  uint32_t edge;   // bit k: step k is on its row's dependency edge
+                   //   (backward: t = T-1, forward: t = 0)
+  bool fast;       // 256-bit (flags: 64-bit) accesses allowed
+  bool few_rows;   // T >= 8: at most one row edge in the tile
+};
+
 // ---------------------------------------------------------------------------
-// Streaming load / store of 4 consecutive steps.  `vec` means the array is
-// 16-byte aligned (4-byte for flags) at every thread's first step, so a single
-// 128-bit (32-bit) access moves all four; otherwise elements are moved one by
-// one.  Steps past the end (k >= nvalid) are neither read nor written.
+// loads / stores of 8 consecutive steps
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void load4(const float *__restrict__ p, uint32_t i0, int nvalid, bool vec,
-                                      float (&v)[4]) {
-  if (vec && nvalid == 4) {
-    float4 t = __ldcs(reinterpret_cast<const float4 *>(p + i0));
-    v[0] = t.x;
-    v[1] = t.y;
-    v[2] = t.z;
-    v[3] = t.w;
+__device__ __forceinline__ void ld8(const float *p, const Tile &tl, float (&v)[8]) {
+  if (tl.fast) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]),
+                   "=f"(v[7])
+                 : "l"(p + tl.i0));
   } else {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) v[k] = k < nvalid ? p[i0 + k] : 0.0f;
+    for (int k = 0; k < 8; ++k) v[k] = k < tl.nvalid ? __ldg(p + tl.i0 + k) : 0.0f;
   }
 }
 
-__device__ __forceinline__ void load4(const int32_t *__restrict__ p, uint32_t i0, int nvalid,
-                                      bool vec, uint32_t (&v)[4]) {
-  if (vec && nvalid == 4) {
-    int4 t = __ldcs(reinterpret_cast<const int4 *>(p + i0));
-    v[0] = uint32_t(t.x);
-    v[1] = uint32_t(t.y);
-    v[2] = uint32_t(t.z);
-    v[3] = uint32_t(t.w);
+__device__ __forceinline__ void ld8(const int32_t *p, const Tile &tl, uint32_t (&v)[8]) {
+  if (tl.fast) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+                   "=r"(v[7])
+                 : "l"(p + tl.i0));
   } else {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) v[k] = k < nvalid ? uint32_t(p[i0 + k]) : 0u;
+    for (int k = 0; k < 8; ++k) v[k] = k < tl.nvalid ? uint32_t(__ldg(p + tl.i0 + k)) : 0u;
   }
 }
 
-// Four flag bytes packed little-endian into one word (byte k = step i0+k).
-__device__ __forceinline__ uint32_t load4_flags(const uint8_t *__restrict__ p, uint32_t i0,
-                                                int nvalid, bool vec) {
+// Bit k set iff byte k of the 8 bytes is nonzero.
+__device__ __forceinline__ uint32_t nonzero_bytes4(uint32_t w) {
+  const uint32_t ones = __vcmpne4(w, 0u) & 0x01010101u;  // bit 8j set iff byte j != 0
+  return ((ones * 0x00204081u) >> 21) & 0xfu;             // gather bits 0, 8, 16, 24
+}
+__device__ __forceinline__ uint32_t ld8_flags(const uint8_t *p, const Tile &tl) {
   if (p == nullptr) return 0u;
-  if (vec && nvalid == 4) return __ldcs(reinterpret_cast<const unsigned int *>(p + i0));
-  uint32_t w = 0;
+  if (tl.fast) {
+    uint32_t lo, hi;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(lo), "=r"(hi) : "l"(p + tl.i0));
+    return nonzero_bytes4(lo) | (nonzero_bytes4(hi) << 4);
+  }
+  uint32_t m = 0;
 #pragma unroll
-  for (int k = 0; k < 4; ++k)
-    if (k < nvalid) w |= uint32_t(p[i0 + k]) << (8 * k);
-  return w;
+  for (int k = 0; k < 8; ++k)
+    if (k < tl.nvalid && __ldg(p + tl.i0 + k) != 0) m |= 1u << k;
+  return m;
 }
 
-__device__ __forceinline__ void store4(float *__restrict__ p, uint32_t i0, int nvalid, bool vec,
-                                       const float (&v)[4]) {
-  if (vec && nvalid == 4) {
-    __stcs(reinterpret_cast<float4 *>(p + i0), make_float4(v[0], v[1], v[2], v[3]));
+__device__ __forceinline__ void st8(float *p, const Tile &tl, const float (&v)[8]) {
+  if (tl.fast) {
+    asm volatile("st.global.cs.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p + tl.i0), "f"(v[0]), "f"(v[1]),
+                 "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+                 : "memory");
   } else {
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      if (k < nvalid) p[i0 + k] = v[k];
+    for (int k = 0; k < 8; ++k)
+      if (k < tl.nvalid) p[tl.i0 + k] = v[k];
   }
 }
 
-__device__ __forceinline__ void store4(int32_t *__restrict__ p, uint32_t i0, int nvalid, bool vec,
-                                       const uint32_t (&v)[4]) {
-  if (vec && nvalid == 4) {
-    __stcs(reinterpret_cast<int4 *>(p + i0),
-           make_int4(int(v[0]), int(v[1]), int(v[2]), int(v[3])));
+__device__ __forceinline__ void st8(int32_t *p, const Tile &tl, const uint32_t (&v)[8]) {
+  if (tl.fast) {
+    asm volatile("st.global.cs.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p + tl.i0), "r"(v[0]), "r"(v[1]),
+                 "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
   } else {
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      if (k < nvalid) p[i0 + k] = int32_t(v[k]);
+    for (int k = 0; k < 8; ++k)
+      if (k < tl.nvalid) p[tl.i0 + k] = int32_t(v[k]);
   }
 }
 
-// Flag bits of step k: bit 0 terminated, bit 1 truncated.
-__device__ __forceinline__ uint32_t step_flags(uint32_t term4, uint32_t trunc4, int k) {
-  return (((term4 >> (8 * k)) & 0xffu) ? 1u : 0u) | (((trunc4 >> (8 * k)) & 0xffu) ? 2u : 0u);
+// Per-row value (bootstrap / initial trace) of the tile's row edge, issued
+// with the tile's other loads: its address follows from the tile position.
+// Tiles of rows shorter than 8 steps (several edges) load theirs in coef().
+__device__ __forceinline__ float edge_value(const float *src, const Tile &tl, const FastDiv &fd) {
+  if (src == nullptr || !tl.few_rows || tl.edge == 0u) return 0.0f;
+  const uint32_t k = __ffs(tl.edge) - 1u;
+  return __ldg(src + tl.n0 + fd.div(tl.t0 + k));
 }
 
-// Successor value of a backward step (boundary semantics).  `next` is the
-// value of step t+1, used only when the step continues inside the window.
-__device__ __forceinline__ float successor_value(uint32_t fl, bool row_end, float next,
-                                                 const float *__restrict__ tv,
-                                                 const float *__restrict__ boot, uint32_t n,
-                                                 uint32_t i, bool &cont) {
-  cont = false;
-  if (fl & 1u) return 0.0f;
-  if (fl & 2u) return __ldg(tv + i);
-  if (row_end) return boot ? __ldg(boot + n) : 0.0f;
-  cont = true;
-  return next;
+// Successor values of the tile's boundary steps (backward estimators): 0 after
+// termination, trunc_value after truncation (the only loads that depend on the
+// data), the row's bootstrap at a row end.
+__device__ __forceinline__ void boundary_values(const float *tv, const float *boot, float edge_val, const Tile &tl,
+                                                uint32_t term, uint32_t trunc, const FastDiv &fd, float (&sv)[8]) {
+  const uint32_t tr = trunc & ~term & tl.valid;
+  const uint32_t ed = tl.edge & ~term & ~trunc;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float s = 0.0f;
+    if ((tr >> k) & 1u)
+      s = __ldg(tv + tl.i0 + k);
+    else if ((ed >> k) & 1u)
+      s = tl.few_rows ? edge_val : (boot ? __ldg(boot + tl.n0 + fd.div(tl.t0 + k)) : 0.0f);
+    sv[k] = s;
+  }
 }
-
-struct NoNbr {};
-struct NoAux {};
 
 // ---------------------------------------------------------------------------
 // GAE (Schulman et al. 2016): x = advantage, a = gamma lambda cont,
@@ -129,45 +152,51 @@ struct NoAux {};
 // ---------------------------------------------------------------------------
 struct GaeOp {
   using V = float;
-  static constexpr bool kBackward = true, kNeedsNbr = true, kPrologue = false;
+  static constexpr bool kBackward = true;
   struct Args {
     const float *r, *v, *boot, *tv;
     const uint8_t *term, *trunc;
     float *adv, *ret;
     float gamma, gl;
   };
-  struct Item {
-    float r, v;
-    uint32_t fl;
+  struct Raw {
+    float r[8], v[8];
+    uint32_t term, trunc;
+    float halo;  // v of the step after the tile (lane 31 only)
+    float ev;    // bootstrap of the tile's row end
   };
-  using Nbr = float;
-  using Aux = NoAux;
-  static __device__ __forceinline__ void load(const Args &p, uint32_t i0, int nv, bool vec,
-                                              Item (&it)[4]) {
-    float r[4], v[4];
-    load4(p.r, i0, nv, vec, r);
-    load4(p.v, i0, nv, vec, v);
-    uint32_t te = load4_flags(p.term, i0, nv, vec), tr = load4_flags(p.trunc, i0, nv, vec);
+  static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int lane,
+                                              uint32_t total, Raw &w) {
+    ld8(p.r, tl, w.r);
+    ld8(p.v, tl, w.v);
+    w.term = ld8_flags(p.term, tl);
+    w.trunc = ld8_flags(p.trunc, tl);
+    w.halo = (lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total) ? __ldg(p.v + tl.i0 + 8u) : 0.0f;
+    w.ev = edge_value(p.boot, tl, fd);
+  }
+  static __device__ __forceinline__ float nbr_of(const Raw &w) { return w.v[0]; }
+  static __device__ __forceinline__ float halo_of(const Raw &w) { return w.halo; }
+  static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w,
+                                              float next7, Aff<float> (&c)[8]) {
+    float sv[8];
+    boundary_values(p.tv, p.boot, w.ev, tl, w.term, w.trunc, fd, sv);
+    const uint32_t special = w.term | w.trunc | tl.edge;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) it[k] = Item{r[k], v[k], step_flags(te, tr, k)};
+    for (int k = 0; k < 8; ++k) {
+      const bool sp = (special >> k) & 1u;
+      const float next = k < 7 ? w.v[k < 7 ? k + 1 : 7] : next7;
+      const float nv = sp ? sv[k] : next;
+      c[k] = Aff<float>{sp ? 0.0f : p.gl, fmaf(p.gamma, nv, w.r[k]) - w.v[k]};
+    }
   }
-  static __device__ __forceinline__ Nbr nbr_of(const Item &it) { return it.v; }
-  static __device__ __forceinline__ Nbr nbr_load(const Args &p, uint32_t i) { return __ldg(p.v + i); }
-  static __device__ __forceinline__ Aff<float> coef(const Args &p, const Item &it, Nbr next,
-                                                    bool row_end, uint32_t n, uint32_t i, Aux &) {
-    bool cont;
-    float nv = successor_value(it.fl, row_end, next, p.tv, p.boot, n, i, cont);
-    return Aff<float>{cont ? p.gl : 0.0f, fmaf(p.gamma, nv, it.r) - it.v};
-  }
-  static __device__ __forceinline__ void emit(const Args &p, uint32_t i0, int nv, bool vec,
-                                              const Item (&it)[4], const float (&x)[4],
-                                              const float (&)[4], const Aux (&)[4]) {
-    store4(p.adv, i0, nv, vec, x);
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &w, const Aff<float> (&)[8],
+                                              const float (&x)[8], const float (&)[8]) {
+    st8(p.adv, tl, x);
     if (p.ret) {
-      float ret[4];
+      float ret[8];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) ret[k] = x[k] + it[k].v;
-      store4(p.ret, i0, nv, vec, ret);
+      for (int k = 0; k < 8; ++k) ret[k] = x[k] + w.v[k];
+      st8(p.ret, tl, ret);
     }
   }
 };
@@ -178,41 +207,44 @@ struct GaeOp {
 // ---------------------------------------------------------------------------
 struct TdLambdaOp {
   using V = float;
-  static constexpr bool kBackward = true, kNeedsNbr = true, kPrologue = false;
+  static constexpr bool kBackward = true;
   struct Args {
     const float *r, *v, *boot, *tv;
     const uint8_t *term, *trunc;
     float *out;
     float gamma, gl, g1l;  // gamma, gamma*lambda, gamma*(1-lambda)
   };
-  struct Item {
-    float r;
-    uint32_t fl;
-    float v;
+  struct Raw {
+    float r[8], v[8];
+    uint32_t term, trunc;
+    float halo, ev;
   };
-  using Nbr = float;
-  using Aux = NoAux;
-  static __device__ __forceinline__ void load(const Args &p, uint32_t i0, int nv, bool vec,
-                                              Item (&it)[4]) {
-    float r[4], v[4];
-    load4(p.r, i0, nv, vec, r);
-    load4(p.v, i0, nv, vec, v);
-    uint32_t te = load4_flags(p.term, i0, nv, vec), tr = load4_flags(p.trunc, i0, nv, vec);
+  static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int lane,
+                                              uint32_t total, Raw &w) {
+    ld8(p.r, tl, w.r);
+    ld8(p.v, tl, w.v);
+    w.term = ld8_flags(p.term, tl);
+    w.trunc = ld8_flags(p.trunc, tl);
+    w.halo = (lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total) ? __ldg(p.v + tl.i0 + 8u) : 0.0f;
+    w.ev = edge_value(p.boot, tl, fd);
+  }
+  static __device__ __forceinline__ float nbr_of(const Raw &w) { return w.v[0]; }
+  static __device__ __forceinline__ float halo_of(const Raw &w) { return w.halo; }
+  static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w,
+                                              float next7, Aff<float> (&c)[8]) {
+    float sv[8];
+    boundary_values(p.tv, p.boot, w.ev, tl, w.term, w.trunc, fd, sv);
+    const uint32_t special = w.term | w.trunc | tl.edge;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) it[k] = Item{r[k], step_flags(te, tr, k), v[k]};
+    for (int k = 0; k < 8; ++k) {
+      const bool sp = (special >> k) & 1u;
+      const float next = k < 7 ? w.v[k < 7 ? k + 1 : 7] : next7;
+      c[k] = sp ? Aff<float>{0.0f, fmaf(p.gamma, sv[k], w.r[k])} : Aff<float>{p.gl, fmaf(p.g1l, next, w.r[k])};
+    }
   }
-  static __device__ __forceinline__ Nbr nbr_of(const Item &it) { return it.v; }
-  static __device__ __forceinline__ Nbr nbr_load(const Args &p, uint32_t i) { return __ldg(p.v + i); }
-  static __device__ __forceinline__ Aff<float> coef(const Args &p, const Item &it, Nbr next,
-                                                    bool row_end, uint32_t n, uint32_t i, Aux &) {
-    bool cont;
-    float nv = successor_value(it.fl, row_end, next, p.tv, p.boot, n, i, cont);
-    return cont ? Aff<float>{p.gl, fmaf(p.g1l, nv, it.r)} : Aff<float>{0.0f, fmaf(p.gamma, nv, it.r)};
-  }
-  static __device__ __forceinline__ void emit(const Args &p, uint32_t i0, int nv, bool vec,
-                                              const Item (&)[4], const float (&x)[4],
-                                              const float (&)[4], const Aux (&)[4]) {
-    store4(p.out, i0, nv, vec, x);
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[8],
+                                              const float (&x)[8], const float (&)[8]) {
+    st8(p.out, tl, x);
   }
 };
 
@@ -222,39 +254,41 @@ struct TdLambdaOp {
 // ---------------------------------------------------------------------------
 struct DiscountedOp {
   using V = float;
-  static constexpr bool kBackward = true, kNeedsNbr = false, kPrologue = false;
+  static constexpr bool kBackward = true;
   struct Args {
     const float *r, *boot, *tv;
     const uint8_t *term, *trunc;
     float *out;
     float gamma;
   };
-  struct Item {
-    float r;
-    uint32_t fl;
+  struct Raw {
+    float r[8];
+    uint32_t term, trunc;
+    float ev;
   };
-  using Nbr = NoNbr;
-  using Aux = NoAux;
-  static __device__ __forceinline__ void load(const Args &p, uint32_t i0, int nv, bool vec,
-                                              Item (&it)[4]) {
-    float r[4];
-    load4(p.r, i0, nv, vec, r);
-    uint32_t te = load4_flags(p.term, i0, nv, vec), tr = load4_flags(p.trunc, i0, nv, vec);
+  static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int, uint32_t,
+                                              Raw &w) {
+    ld8(p.r, tl, w.r);
+    w.term = ld8_flags(p.term, tl);
+    w.trunc = ld8_flags(p.trunc, tl);
+    w.ev = edge_value(p.boot, tl, fd);
+  }
+  static __device__ __forceinline__ float nbr_of(const Raw &) { return 0.0f; }
+  static __device__ __forceinline__ float halo_of(const Raw &) { return 0.0f; }
+  static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w, float,
+                                              Aff<float> (&c)[8]) {
+    float sv[8];
+    boundary_values(p.tv, p.boot, w.ev, tl, w.term, w.trunc, fd, sv);
+    const uint32_t special = w.term | w.trunc | tl.edge;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) it[k] = Item{r[k], step_flags(te, tr, k)};
+    for (int k = 0; k < 8; ++k) {
+      const bool sp = (special >> k) & 1u;
+      c[k] = sp ? Aff<float>{0.0f, fmaf(p.gamma, sv[k], w.r[k])} : Aff<float>{p.gamma, w.r[k]};
+    }
   }
-  static __device__ __forceinline__ Nbr nbr_of(const Item &) { return NoNbr{}; }
-  static __device__ __forceinline__ Nbr nbr_load(const Args &, uint32_t) { return NoNbr{}; }
-  static __device__ __forceinline__ Aff<float> coef(const Args &p, const Item &it, Nbr,
-                                                    bool row_end, uint32_t n, uint32_t i, Aux &) {
-    bool cont;
-    float nv = successor_value(it.fl, row_end, 0.0f, p.tv, p.boot, n, i, cont);
-    return cont ? Aff<float>{p.gamma, it.r} : Aff<float>{0.0f, fmaf(p.gamma, nv, it.r)};
-  }
-  static __device__ __forceinline__ void emit(const Args &p, uint32_t i0, int nv, bool vec,
-                                              const Item (&)[4], const float (&x)[4],
-                                              const float (&)[4], const Aux (&)[4]) {
-    store4(p.out, i0, nv, vec, x);
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[8],
+                                              const float (&x)[8], const float (&)[8]) {
+    st8(p.out, tl, x);
   }
 };
 
@@ -262,62 +296,62 @@ struct DiscountedOp {
 // V-trace (Espeholt et al. 2018) with lambda-scaled traces, on d = vs - v:
 // rho = min(rho_bar, e^lr), c = lambda min(c_bar, e^lr),
 // a = gamma c cont, b = rho (r + gamma nv - v).  Outputs vs = x + v and
-// pg_adv = rho (r + gamma (nv + [cont] x_{t+1}) - v), since vs_{t+1} =
-// v_{t+1} + d_{t+1} inside an episode and nv at a boundary.
+// pg_adv = b + gamma rho cont x_{t+1}: rho (r + gamma vs_{t+1} - v) inside an
+// episode (vs_{t+1} = v_{t+1} + x_{t+1}), rho (r + gamma nv - v) at a boundary.
 // ---------------------------------------------------------------------------
 struct VtraceOp {
   using V = float;
-  static constexpr bool kBackward = true, kNeedsNbr = true, kPrologue = false;
+  static constexpr bool kBackward = true;
   struct Args {
     const float *lr, *r, *v, *boot, *tv;
     const uint8_t *term, *trunc;
     float *vs, *pg;
     float gamma, lambda, rho_bar, c_bar;
   };
-  struct Item {
-    float lr, r, v;
-    uint32_t fl;
+  struct Raw {
+    float lr[8], r[8], v[8];  // coef() keeps gamma * rho * cont in lr for emit()
+    uint32_t term, trunc;
+    float halo, ev;
   };
-  using Nbr = float;
-  struct Aux {
-    float rho, nv, contf;
-  };
-  static __device__ __forceinline__ void load(const Args &p, uint32_t i0, int nv, bool vec,
-                                              Item (&it)[4]) {
-    float lr[4], r[4], v[4];
-    load4(p.lr, i0, nv, vec, lr);
-    load4(p.r, i0, nv, vec, r);
-    load4(p.v, i0, nv, vec, v);
-    uint32_t te = load4_flags(p.term, i0, nv, vec), tr = load4_flags(p.trunc, i0, nv, vec);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) it[k] = Item{lr[k], r[k], v[k], step_flags(te, tr, k)};
+  static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int lane,
+                                              uint32_t total, Raw &w) {
+    ld8(p.lr, tl, w.lr);
+    ld8(p.r, tl, w.r);
+    ld8(p.v, tl, w.v);
+    w.term = ld8_flags(p.term, tl);
+    w.trunc = ld8_flags(p.trunc, tl);
+    w.halo = (lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total) ? __ldg(p.v + tl.i0 + 8u) : 0.0f;
+    w.ev = edge_value(p.boot, tl, fd);
   }
-  static __device__ __forceinline__ Nbr nbr_of(const Item &it) { return it.v; }
-  static __device__ __forceinline__ Nbr nbr_load(const Args &p, uint32_t i) { return __ldg(p.v + i); }
-  static __device__ __forceinline__ Aff<float> coef(const Args &p, const Item &it, Nbr next,
-                                                    bool row_end, uint32_t n, uint32_t i,
-                                                    Aux &aux) {
-    bool cont;
-    float nv = successor_value(it.fl, row_end, next, p.tv, p.boot, n, i, cont);
-    float ratio = expf(it.lr);
-    float rho = fminf(p.rho_bar, ratio);
-    float c = p.lambda * fminf(p.c_bar, ratio);
-    aux = Aux{rho, nv, cont ? 1.0f : 0.0f};
-    return Aff<float>{cont ? p.gamma * c : 0.0f, rho * (fmaf(p.gamma, nv, it.r) - it.v)};
-  }
-  static __device__ __forceinline__ void emit(const Args &p, uint32_t i0, int nv, bool vec,
-                                              const Item (&it)[4], const float (&x)[4],
-                                              const float (&xn)[4], const Aux (&aux)[4]) {
-    float vs[4];
+  static __device__ __forceinline__ float nbr_of(const Raw &w) { return w.v[0]; }
+  static __device__ __forceinline__ float halo_of(const Raw &w) { return w.halo; }
+  static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w,
+                                              float next7, Aff<float> (&c)[8]) {
+    float sv[8];
+    boundary_values(p.tv, p.boot, w.ev, tl, w.term, w.trunc, fd, sv);
+    const uint32_t special = w.term | w.trunc | tl.edge;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) vs[k] = x[k] + it[k].v;
-    store4(p.vs, i0, nv, vec, vs);
+    for (int k = 0; k < 8; ++k) {
+      const bool sp = (special >> k) & 1u;
+      const float next = k < 7 ? w.v[k < 7 ? k + 1 : 7] : next7;
+      const float nv = sp ? sv[k] : next;
+      const float ratio = __expf(w.lr[k]);
+      const float rho = fminf(p.rho_bar, ratio);
+      const float cc = p.lambda * fminf(p.c_bar, ratio);
+      c[k] = Aff<float>{sp ? 0.0f : p.gamma * cc, rho * (fmaf(p.gamma, nv, w.r[k]) - w.v[k])};
+      w.lr[k] = sp ? 0.0f : p.gamma * rho;
+    }
+  }
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &w, const Aff<float> (&c)[8],
+                                              const float (&x)[8], const float (&xn)[8]) {
+    float o[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) o[k] = x[k] + w.v[k];
+    st8(p.vs, tl, o);
     if (p.pg) {
-      float pg[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        pg[k] = aux[k].rho * (fmaf(p.gamma, fmaf(aux[k].contf, xn[k], aux[k].nv), it[k].r) - it[k].v);
-      store4(p.pg, i0, nv, vec, pg);
+      for (int k = 0; k < 8; ++k) o[k] = fmaf(w.lr[k], xn[k], c[k].b);
+      st8(p.pg, tl, o);
     }
   }
 };
@@ -329,40 +363,44 @@ struct VtraceOp {
 // ---------------------------------------------------------------------------
 struct EligOp {
   using V = float;
-  static constexpr bool kBackward = false, kNeedsNbr = true, kPrologue = false;
+  static constexpr bool kBackward = false;
   struct Args {
     const float *g, *init;
     const uint8_t *term, *trunc;
     float *out;
     float gl;
   };
-  struct Item {
-    float g;
-    uint32_t fl;
+  struct Raw {
+    float g[8];
+    uint32_t done;  // bit k: step k terminated or truncated
+    uint32_t halo;  // done flag of the step before the tile (lane 0 only)
+    float ev;       // initial trace of the tile's row start
   };
-  using Nbr = uint32_t;  // previous step done (0/1)
-  using Aux = NoAux;
-  static __device__ __forceinline__ void load(const Args &p, uint32_t i0, int nv, bool vec,
-                                              Item (&it)[4]) {
-    float g[4];
-    load4(p.g, i0, nv, vec, g);
-    uint32_t te = load4_flags(p.term, i0, nv, vec), tr = load4_flags(p.trunc, i0, nv, vec);
+  static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int lane, uint32_t,
+                                              Raw &w) {
+    ld8(p.g, tl, w.g);
+    w.done = ld8_flags(p.term, tl) | ld8_flags(p.trunc, tl);
+    w.halo = 0u;
+    if (lane == 0 && tl.i0 > 0u && tl.nvalid > 0)
+      w.halo = ((p.term && __ldg(p.term + tl.i0 - 1u)) || (p.trunc && __ldg(p.trunc + tl.i0 - 1u))) ? 1u : 0u;
+    w.ev = edge_value(p.init, tl, fd);
+  }
+  static __device__ __forceinline__ uint32_t nbr_of(const Raw &w) { return (w.done >> 7) & 1u; }
+  static __device__ __forceinline__ uint32_t halo_of(const Raw &w) { return w.halo; }
+  static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w,
+                                              uint32_t prev7, Aff<float> (&c)[8]) {
+    const uint32_t cut = (((w.done << 1) | prev7) | tl.edge) & 0xffu;  // bit k: a_k = 0
 #pragma unroll
-    for (int k = 0; k < 4; ++k) it[k] = Item{g[k], step_flags(te, tr, k)};
+    for (int k = 0; k < 8; ++k) {
+      float b = w.g[k];
+      if (((tl.edge >> k) & 1u) && p.init)
+        b = fmaf(p.gl, tl.few_rows ? w.ev : __ldg(p.init + tl.n0 + fd.div(tl.t0 + k)), b);
+      c[k] = Aff<float>{((cut >> k) & 1u) ? 0.0f : p.gl, b};
+    }
   }
-  static __device__ __forceinline__ Nbr nbr_of(const Item &it) { return it.fl ? 1u : 0u; }
-  static __device__ __forceinline__ Nbr nbr_load(const Args &p, uint32_t i) {
-    return ((p.term != nullptr && p.term[i] != 0) || (p.trunc != nullptr && p.trunc[i] != 0)) ? 1u : 0u;
-  }
-  static __device__ __forceinline__ Aff<float> coef(const Args &p, const Item &it, Nbr prev_done,
-                                                    bool row_start, uint32_t n, uint32_t, Aux &) {
-    if (row_start) return Aff<float>{0.0f, p.init ? fmaf(p.gl, __ldg(p.init + n), it.g) : it.g};
-    return Aff<float>{prev_done ? 0.0f : p.gl, it.g};
-  }
-  static __device__ __forceinline__ void emit(const Args &p, uint32_t i0, int nv, bool vec,
-                                              const Item (&)[4], const float (&x)[4],
-                                              const float (&)[4], const Aux (&)[4]) {
-    store4(p.out, i0, nv, vec, x);
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[8],
+                                              const float (&x)[8], const float (&)[8]) {
+    st8(p.out, tl, x);
   }
 };
 
@@ -372,38 +410,36 @@ struct EligOp {
 // ---------------------------------------------------------------------------
 struct PrefixSumOp {
   using V = uint32_t;
-  static constexpr bool kBackward = false, kNeedsNbr = true, kPrologue = false;
+  static constexpr bool kBackward = false;
   struct Args {
     const int32_t *x;
     const uint8_t *term, *trunc;
     int32_t *out;
   };
-  struct Item {
-    uint32_t x;
-    uint32_t fl;
+  struct Raw {
+    uint32_t x[8];
+    uint32_t done;
+    uint32_t halo;
   };
-  using Nbr = uint32_t;
-  using Aux = NoAux;
-  static __device__ __forceinline__ void load(const Args &p, uint32_t i0, int nv, bool vec,
-                                              Item (&it)[4]) {
-    uint32_t x[4];
-    load4(p.x, i0, nv, vec, x);
-    uint32_t te = load4_flags(p.term, i0, nv, vec), tr = load4_flags(p.trunc, i0, nv, vec);
+  static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &, int lane, uint32_t,
+                                              Raw &w) {
+    ld8(p.x, tl, w.x);
+    w.done = ld8_flags(p.term, tl) | ld8_flags(p.trunc, tl);
+    w.halo = 0u;
+    if (lane == 0 && tl.i0 > 0u && tl.nvalid > 0)
+      w.halo = ((p.term && __ldg(p.term + tl.i0 - 1u)) || (p.trunc && __ldg(p.trunc + tl.i0 - 1u))) ? 1u : 0u;
+  }
+  static __device__ __forceinline__ uint32_t nbr_of(const Raw &w) { return (w.done >> 7) & 1u; }
+  static __device__ __forceinline__ uint32_t halo_of(const Raw &w) { return w.halo; }
+  static __device__ __forceinline__ void coef(const Args &, const Tile &tl, const FastDiv &, Raw &w, uint32_t prev7,
+                                              Aff<uint32_t> (&c)[8]) {
+    const uint32_t cut = (((w.done << 1) | prev7) | tl.edge) & 0xffu;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) it[k] = Item{x[k], step_flags(te, tr, k)};
+    for (int k = 0; k < 8; ++k) c[k] = Aff<uint32_t>{((cut >> k) & 1u) ^ 1u, w.x[k]};
   }
-  static __device__ __forceinline__ Nbr nbr_of(const Item &it) { return it.fl ? 1u : 0u; }
-  static __device__ __forceinline__ Nbr nbr_load(const Args &p, uint32_t i) {
-    return ((p.term != nullptr && p.term[i] != 0) || (p.trunc != nullptr && p.trunc[i] != 0)) ? 1u : 0u;
-  }
-  static __device__ __forceinline__ Aff<uint32_t> coef(const Args &, const Item &it, Nbr prev_done,
-                                                       bool row_start, uint32_t, uint32_t, Aux &) {
-    return Aff<uint32_t>{(row_start || prev_done) ? 0u : 1u, it.x};
-  }
-  static __device__ __forceinline__ void emit(const Args &p, uint32_t i0, int nv, bool vec,
-                                              const Item (&)[4], const uint32_t (&x)[4],
-                                              const uint32_t (&)[4], const Aux (&)[4]) {
-    store4(p.out, i0, nv, vec, x);
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<uint32_t> (&)[8],
+                                              const uint32_t (&x)[8], const uint32_t (&)[8]) {
+    st8(p.out, tl, x);
   }
 };
 

@@ -19,66 +19,67 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "async_copy.cuh"
 #include "estimators.cuh"
 #include "scan_core.cuh"
+#include "scan_kernel.cuh"
 
 namespace rlscan {
 
-__device__ __forceinline__ uint32_t smem_addr(const void *p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
-               : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Global -> shared bulk copy (no tensor map, no multicast); `bytes` is a
-// multiple of 16 and both addresses are 16-byte aligned.
-__device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes,
-                                              uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
+// 4 consecutive steps per thread (128-bit accesses when aligned).
+__device__ __forceinline__ void load4(const float *__restrict__ p, uint32_t i0, int nvalid, bool vec,
+                                      float (&v)[4]) {
+  if (vec && nvalid == 4) {
+    float4 t = __ldcs(reinterpret_cast<const float4 *>(p + i0));
+    v[0] = t.x;
+    v[1] = t.y;
+    v[2] = t.z;
+    v[3] = t.w;
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = k < nvalid ? p[i0 + k] : 0.0f;
+  }
 }
 
-// Bounded wait for an mbarrier phase: gives up after `timeout_ns` of global
-// time, recording the timeout status (the block then carries on with whatever
-// the buffer holds, so it neither hangs nor traps).
-__device__ __forceinline__ void mbar_wait_bounded(uint64_t *bar, uint32_t parity,
-                                                  uint64_t timeout_ns) {
-  if (mbar_try_wait(bar, parity)) return;
-  const uint64_t t0 = global_timer_ns();
-  uint64_t iters = 0;
-  const uint64_t max_iters = 64 + timeout_ns / 16;
-  while (!mbar_try_wait(bar, parity)) {
-    if (++iters > max_iters || global_timer_ns() - t0 > timeout_ns) {
-      record_status(kDevStatusTimeout);
-      return;
-    }
+// Four flag bytes packed little-endian into one word (byte k = step i0+k).
+__device__ __forceinline__ uint32_t load4_flags(const uint8_t *__restrict__ p, uint32_t i0, int nvalid,
+                                                bool vec) {
+  if (p == nullptr) return 0u;
+  if (vec && nvalid == 4) return __ldcs(reinterpret_cast<const unsigned int *>(p + i0));
+  uint32_t w = 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    if (k < nvalid) w |= uint32_t(p[i0 + k]) << (8 * k);
+  return w;
+}
+
+__device__ __forceinline__ void store4(float *__restrict__ p, uint32_t i0, int nvalid, bool vec,
+                                       const float (&v)[4]) {
+  if (vec && nvalid == 4) {
+    __stcs(reinterpret_cast<float4 *>(p + i0), make_float4(v[0], v[1], v[2], v[3]));
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k < nvalid) p[i0 + k] = v[k];
   }
+}
+
+// Flag bits of step k: bit 0 terminated, bit 1 truncated.
+__device__ __forceinline__ uint32_t step_flags(uint32_t term4, uint32_t trunc4, int k) {
+  return (((term4 >> (8 * k)) & 0xffu) ? 1u : 0u) | (((trunc4 >> (8 * k)) & 0xffu) ? 2u : 0u);
+}
+
+// Successor value of a backward step (boundary semantics).
+__device__ __forceinline__ float successor_value(uint32_t fl, bool row_end, float next,
+                                                 const float *__restrict__ tv,
+                                                 const float *__restrict__ boot, uint32_t n,
+                                                 uint32_t i, bool &cont) {
+  cont = false;
+  if (fl & 1u) return 0.0f;
+  if (fl & 2u) return __ldg(tv + i);
+  if (row_end) return boot ? __ldg(boot + n) : 0.0f;
+  cont = true;
+  return next;
 }
 
 struct RetraceOp {
@@ -102,7 +103,7 @@ struct RetraceOp {
   struct Nbr {
     float e, qa, c;
   };
-  using Aux = NoAux;
+  struct Aux {};
 
   // Dynamic shared memory layout for a chunk of L steps:
   //   float E[L + 1], Qa[L + 1], C[L + 1]   (index L: first step after the chunk)
@@ -273,5 +274,115 @@ struct RetraceOp {
     }
   }
 };
+
+// One block per chunk of L = 4 * BLOCK steps: the prologue fills E, q_a, c
+// for the chunk (and the step after it) in shared memory, then each thread
+// scans 4 consecutive steps; warps and blocks combine as in scan_kernel.cuh.
+// With LB, blocks take tickets in dependency order (one per block) and chain
+// carries with the decoupled look-back.
+template <int BLOCK, bool LB>
+__global__ void __launch_bounds__(BLOCK) retrace_kernel(const RetraceOp::Args p, const ScanGeom g) {
+  using Op = RetraceOp;
+  using V = float;
+  using Item = Op::Item;
+  using Nbr = Op::Nbr;
+  using Aux = Op::Aux;
+  constexpr int W = BLOCK / 32;
+  constexpr uint32_t L = 4u * BLOCK;
+  __shared__ Aff<V> s_wagg[W];
+  __shared__ V s_wcarry[W];
+  __shared__ uint32_t s_ticket, s_epoch;
+  extern __shared__ __align__(16) unsigned char dyn_smem[];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const FastDiv fd{g.div_m, g.div_l};
+  uint32_t chunk = blockIdx.x, ticket = 0, epoch = 0;
+  if constexpr (LB) {
+    if (tid == 0) {
+      s_ticket = atomicInc(&g.lb.hdr->ticket, g.fetch_wrap);
+      s_epoch = *reinterpret_cast<volatile uint32_t *>(&g.lb.hdr->epoch);
+    }
+    __syncthreads();
+    ticket = s_ticket;
+    epoch = s_epoch;
+    if (ticket >= g.nchunks) {  // counter left inconsistent by an aborted launch
+      if (tid == 0) record_status(kDevStatusTimeout);
+      return;
+    }
+    chunk = g.nchunks - 1u - ticket;
+  }
+  const uint32_t cbase = chunk * L;
+  Op::prologue(p, cbase, L, g.total, dyn_smem, tid, BLOCK, g.lb.timeout_ns);
+
+  const uint32_t i0 = cbase + 4u * uint32_t(tid);
+  const int nvalid = i0 < g.total ? int(min(4u, g.total - i0)) : 0;
+  uint32_t n = 0, t = 0;
+  if (nvalid) {
+    n = fd.div(i0);
+    t = i0 - n * g.T;
+  }
+  Item it[4];
+  Op::load(p, i0, nvalid, g.vec != 0u, it);
+  Nbr nb[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) nb[k] = Op::nbr_smem(dyn_smem, L, 4u * uint32_t(tid) + k + 1u);
+
+  Aff<V> c[4];
+  Aux aux[4] = {};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if (k < nvalid)
+      c[k] = Op::coef(p, it[k], nb[k], t == g.T - 1u, n, i0 + k, aux[k]);
+    else
+      c[k] = aff_identity<V>();
+    if (++t == g.T) {
+      t = 0;
+      ++n;
+    }
+  }
+  Aff<V> agg = compose(c[2], c[3]);
+  agg = compose(c[1], agg);
+  agg = compose(c[0], agg);
+
+  const Aff<V> inc = warp_inclusive_scan<true>(agg, lane);
+  const Aff<V> exc = warp_exclusive_from_inclusive<true>(inc, lane, 31);
+  if (lane == 0) s_wagg[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    const Aff<V> wv = lane < W ? s_wagg[lane] : aff_identity<V>();
+    const Aff<V> winc = warp_inclusive_scan<true>(wv, lane);
+    const Aff<V> wexc = warp_exclusive_from_inclusive<true>(winc, lane, W - 1);
+    V carry = 0.0f;
+    if constexpr (LB) {
+      const V ca = __shfl_sync(0xffffffffu, winc.a, 0);
+      const V cb = __shfl_sync(0xffffffffu, winc.b, 0);
+      if (lane == 0) {
+        const bool edge_closed = (min(cbase + L, g.total) % g.T) == 0u;
+        carry = decoupled_lookback<true, V>(g.lb, chunk, g.nchunks, epoch, ticket, Aff<V>{ca, cb},
+                                            edge_closed);
+      }
+      carry = __shfl_sync(0xffffffffu, carry, 0);
+    }
+    if (lane < W) s_wcarry[lane] = apply(wexc, carry);
+  }
+  __syncthreads();
+
+  V x = apply(exc, s_wcarry[warp]);
+  V xs[4], xd[4];
+#pragma unroll
+  for (int k = 3; k >= 0; --k) {
+    xd[k] = x;
+    x = apply(c[k], x);
+    xs[k] = x;
+  }
+  Op::emit(p, i0, nvalid, g.vec != 0u, it, xs, xd, aux);
+
+  if constexpr (LB) {
+    if (tid == 0) {
+      __threadfence();
+      if (atomicInc(&g.lb.hdr->done, g.nchunks - 1u) == g.nchunks - 1u) atomicAdd(&g.lb.hdr->epoch, 1u);
+    }
+  }
+}
 
 }  // namespace rlscan

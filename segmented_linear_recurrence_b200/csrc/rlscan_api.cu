@@ -11,6 +11,7 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 #include <vector>
 
@@ -182,48 +183,50 @@ bool aligned(const void *p, uintptr_t a) { return p == nullptr || reinterpret_ca
 // ---------------------------------------------------------------------------
 struct Plan {
   int block = 256;
-  uint32_t L = 1024;
+  uint32_t L = 2048;        // steps per chunk
   bool lookback = false;
   int64_t rows_per_launch = 0;
   int launches = 0;
-  int64_t blocks = 0;
-  uint32_t max_chunks = 0;
+  int64_t chunks = 0;       // over all launches
+  uint32_t max_chunks = 0;  // in one launch
   size_t ws_bytes = 0;
   // Retrace staging
   uint32_t sub_steps = 0, stages = 0;
   size_t smem = 0;
 };
 
-bool valid_block(int64_t b) { return b == 128 || b == 256 || b == 512 || b == 1024; }
+bool valid_block(int64_t b) { return b == 128 || b == 256 || b == 512; }
 
 Plan make_plan(rlscan_estimator est, int64_t N, int64_t T, int64_t A) {
   Plan pl;
   const int64_t fb = g_force_block.load();
   if (est == RLSCAN_EST_RETRACE) {
     pl.block = (fb == 128 || fb == 256) ? int(fb) : 128;
-  } else if (valid_block(fb)) {
-    pl.block = int(fb);
+    pl.L = 4u * uint32_t(pl.block);
   } else {
-    pl.block = 0;
-    for (int b : {256, 512, 1024})
-      if ((4 * int64_t(b)) % T == 0) {
-        pl.block = b;
-        break;
-      }
-    if (pl.block == 0) pl.block = 512;
+    if (valid_block(fb)) {
+      pl.block = int(fb);
+    } else {
+      pl.block = 0;
+      for (int b : {128, 256, 512})
+        if ((int64_t(kTile) * b) % T == 0) {
+          pl.block = b;
+          break;
+        }
+      if (pl.block == 0) pl.block = 256;
+    }
+    pl.L = uint32_t(kTile) * uint32_t(pl.block);
   }
-  pl.L = 4u * uint32_t(pl.block);
   pl.lookback = g_force_lookback.load() != 0 || (int64_t(pl.L) % T) != 0;
   pl.rows_per_launch = std::max<int64_t>(1, kMaxStepsPerLaunch / T);
   pl.launches = int((N + pl.rows_per_launch - 1) / pl.rows_per_launch);
-  pl.blocks = 0;
   for (int64_t r0 = 0; r0 < N; r0 += pl.rows_per_launch) {
     const int64_t rows = std::min(pl.rows_per_launch, N - r0);
     const uint32_t nch = uint32_t((rows * T + pl.L - 1) / pl.L);
-    pl.blocks += nch;
+    pl.chunks += nch;
     pl.max_chunks = std::max(pl.max_chunks, nch);
   }
-  pl.ws_bytes = pl.lookback ? sizeof(LookbackHeader) + size_t(pl.max_chunks) * sizeof(LookbackDesc) : 0;
+  pl.ws_bytes = sizeof(LookbackHeader) + (pl.lookback ? size_t(pl.max_chunks) * sizeof(LookbackDesc) : 0);
   if (est == RLSCAN_EST_RETRACE) {
     // Sub-tile steps and ring depth: the largest staging that keeps at least
     // three blocks resident per SM (<= ~72 KB of shared memory each).
@@ -239,51 +242,65 @@ Plan make_plan(rlscan_estimator est, int64_t N, int64_t T, int64_t A) {
   return pl;
 }
 
-template <class Op, int BLOCK, bool LB>
-cudaError_t launch_kernel(const typename Op::Args &a, const ScanGeom &g, size_t smem,
-                          cudaStream_t s) {
-  auto kern = scan_kernel<Op, BLOCK, LB>;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
+// (m, l) of FastDiv for divisor d (1 <= d <= 2^30).
+void fast_div_params(uint32_t d, uint32_t &m, uint32_t &l) {
+  if (d <= 1) {
+    m = 0;
+    l = 0;
+    return;
   }
-  kern<<<g.nchunks, BLOCK, smem, s>>>(a, g);
+  l = 0;
+  while ((uint64_t(1) << l) < d) ++l;
+  m = uint32_t(((uint64_t(1) << (31 + l)) + d - 1) / d);
+}
+
+template <class Op, int BLOCK, bool LB>
+cudaError_t launch_scan(const typename Op::Args &a, ScanGeom g, cudaStream_t s) {
+  g.fetch_wrap = g.nchunks - 1u;  // one ticket per block
+  scan_kernel<Op, BLOCK, LB><<<g.nchunks, BLOCK, 0, s>>>(a, g);
   return cudaGetLastError();
 }
 
 template <class Op>
-cudaError_t launch_block(const typename Op::Args &a, const ScanGeom &g, int block, bool lb,
-                         size_t smem, cudaStream_t s) {
+cudaError_t launch_block(const typename Op::Args &a, const ScanGeom &g, int block, bool lb, cudaStream_t s) {
   switch (block) {
-    case 128: return lb ? launch_kernel<Op, 128, true>(a, g, smem, s) : launch_kernel<Op, 128, false>(a, g, smem, s);
-    case 256: return lb ? launch_kernel<Op, 256, true>(a, g, smem, s) : launch_kernel<Op, 256, false>(a, g, smem, s);
-    case 512: return lb ? launch_kernel<Op, 512, true>(a, g, smem, s) : launch_kernel<Op, 512, false>(a, g, smem, s);
-    case 1024: return lb ? launch_kernel<Op, 1024, true>(a, g, smem, s) : launch_kernel<Op, 1024, false>(a, g, smem, s);
+    case 128: return lb ? launch_scan<Op, 128, true>(a, g, s) : launch_scan<Op, 128, false>(a, g, s);
+    case 256: return lb ? launch_scan<Op, 256, true>(a, g, s) : launch_scan<Op, 256, false>(a, g, s);
+    case 512: return lb ? launch_scan<Op, 512, true>(a, g, s) : launch_scan<Op, 512, false>(a, g, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <class Op>
-cudaError_t launch_block_retrace(const typename Op::Args &a, const ScanGeom &g, int block, bool lb,
-                                 size_t smem, cudaStream_t s) {
+template <int BLOCK, bool LB>
+cudaError_t launch_retrace(const RetraceOp::Args &a, ScanGeom g, size_t smem, cudaStream_t s) {
+  auto kern = retrace_kernel<BLOCK, LB>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+  }
+  g.fetch_wrap = g.nchunks - 1u;
+  kern<<<g.nchunks, BLOCK, smem, s>>>(a, g);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_retrace_block(const RetraceOp::Args &a, const ScanGeom &g, int block, bool lb, size_t smem,
+                                 cudaStream_t s) {
   switch (block) {
-    case 128: return lb ? launch_kernel<Op, 128, true>(a, g, smem, s) : launch_kernel<Op, 128, false>(a, g, smem, s);
-    case 256: return lb ? launch_kernel<Op, 256, true>(a, g, smem, s) : launch_kernel<Op, 256, false>(a, g, smem, s);
+    case 128: return lb ? launch_retrace<128, true>(a, g, smem, s) : launch_retrace<128, false>(a, g, smem, s);
+    case 256: return lb ? launch_retrace<256, true>(a, g, smem, s) : launch_retrace<256, false>(a, g, smem, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-// Runs every row slice of a call.  `make_args(row0, vec)` returns the
-// estimator's arguments with every pointer advanced to row `row0`; `slice_vec`
+// Runs every row slice of a call.  `make_args(row0)` returns the estimator's
+// arguments with every pointer advanced to row `row0`; `slice_vec(row0)`
 // tells whether that slice's pointers allow vectorised access.
 template <class Op, class MakeArgs, class SliceVec>
 rlscan_status run(const Plan &pl, int64_t N, int64_t T, rlscan_stream_t stream, MakeArgs make_args,
                   SliceVec slice_vec) {
   void *ws = nullptr;
-  if (pl.lookback) {
-    rlscan_status s = get_workspace(stream, pl.ws_bytes, &ws);
-    if (s != RLSCAN_OK) return s;
-  }
+  rlscan_status st = get_workspace(stream, pl.ws_bytes, &ws);
+  if (st != RLSCAN_OK) return st;
   for (int64_t r0 = 0; r0 < N; r0 += pl.rows_per_launch) {
     const int64_t rows = std::min(pl.rows_per_launch, N - r0);
     ScanGeom g{};
@@ -292,16 +309,17 @@ rlscan_status run(const Plan &pl, int64_t N, int64_t T, rlscan_stream_t stream, 
     g.nchunks = uint32_t((rows * T + pl.L - 1) / pl.L);
     const bool vec = g_force_scalar.load() == 0 && slice_vec(r0);
     g.vec = vec ? 1u : 0u;
+    fast_div_params(uint32_t(T), g.div_m, g.div_l);
     g.lb.hdr = static_cast<LookbackHeader *>(ws);
-    g.lb.desc = ws ? reinterpret_cast<LookbackDesc *>(static_cast<LookbackHeader *>(ws) + 1) : nullptr;
+    g.lb.desc = reinterpret_cast<LookbackDesc *>(static_cast<LookbackHeader *>(ws) + 1);
     g.lb.timeout_ns = uint64_t(std::max<int64_t>(1000, g_timeout_ns.load()));
     g.lb.starve = g_starve.load() != 0 ? 1u : 0u;
-    const typename Op::Args a = make_args(r0, vec);
+    const typename Op::Args a = make_args(r0);
     cudaError_t e;
-    if constexpr (Op::kPrologue)
-      e = launch_block_retrace<Op>(a, g, pl.block, pl.lookback, pl.smem, stream);
+    if constexpr (std::is_same<Op, RetraceOp>::value)
+      e = launch_retrace_block(a, g, pl.block, pl.lookback, pl.smem, stream);
     else
-      e = launch_block<Op>(a, g, pl.block, pl.lookback, 0, stream);
+      e = launch_block<Op>(a, g, pl.block, pl.lookback, stream);
     if (e != cudaSuccess) return RLSCAN_ERR_LAUNCH;
   }
   return RLSCAN_OK;
@@ -341,7 +359,7 @@ rlscan_status rlscan_gae(const float *rewards, const float *values, const float 
   const float *tv = truncated ? trunc_value : nullptr;
   return run<GaeOp>(
       pl, N, T, stream,
-      [&](int64_t r0, bool) {
+      [&](int64_t r0) {
         const int64_t o = r0 * T;
         return GaeOp::Args{adv(rewards, o), adv(values, o), adv(bootstrap, r0), adv(tv, o),
                            adv(terminated, o), adv(truncated, o), adv(advantages, o), adv(returns, o),
@@ -349,9 +367,9 @@ rlscan_status rlscan_gae(const float *rewards, const float *values, const float 
       },
       [&](int64_t r0) {
         const int64_t o = r0 * T;
-        return aligned(adv(rewards, o), 16) && aligned(adv(values, o), 16) &&
-               aligned(adv(advantages, o), 16) && aligned(adv(returns, o), 16) &&
-               aligned(adv(terminated, o), 4) && aligned(adv(truncated, o), 4);
+        return aligned(adv(rewards, o), 32) && aligned(adv(values, o), 32) &&
+               aligned(adv(advantages, o), 32) && aligned(adv(returns, o), 32) &&
+               aligned(adv(terminated, o), 8) && aligned(adv(truncated, o), 8);
       });
 }
 
@@ -378,7 +396,7 @@ rlscan_status rlscan_vtrace(const float *log_rhos, const float *rewards, const f
   const float *tv = truncated ? trunc_value : nullptr;
   return run<VtraceOp>(
       pl, N, T, stream,
-      [&](int64_t r0, bool) {
+      [&](int64_t r0) {
         const int64_t o = r0 * T;
         return VtraceOp::Args{adv(log_rhos, o), adv(rewards, o), adv(values, o), adv(bootstrap, r0),
                               adv(tv, o), adv(terminated, o), adv(truncated, o), adv(vs, o),
@@ -386,10 +404,10 @@ rlscan_status rlscan_vtrace(const float *log_rhos, const float *rewards, const f
       },
       [&](int64_t r0) {
         const int64_t o = r0 * T;
-        return aligned(adv(log_rhos, o), 16) && aligned(adv(rewards, o), 16) &&
-               aligned(adv(values, o), 16) && aligned(adv(vs, o), 16) &&
-               aligned(adv(pg_advantages, o), 16) && aligned(adv(terminated, o), 4) &&
-               aligned(adv(truncated, o), 4);
+        return aligned(adv(log_rhos, o), 32) && aligned(adv(rewards, o), 32) &&
+               aligned(adv(values, o), 32) && aligned(adv(vs, o), 32) &&
+               aligned(adv(pg_advantages, o), 32) && aligned(adv(terminated, o), 8) &&
+               aligned(adv(truncated, o), 8);
       });
 }
 
@@ -418,7 +436,7 @@ rlscan_status rlscan_retrace(const float *q, const float *pi, const float *mu_a,
   const float *tv = truncated ? trunc_value : nullptr;
   return run<RetraceOp>(
       pl, N, T, stream,
-      [&](int64_t r0, bool) {
+      [&](int64_t r0) {
         const int64_t o = r0 * T;
         const int64_t oa = o * A;
         RetraceOp::Args a{};
@@ -459,7 +477,7 @@ rlscan_status rlscan_td_lambda(const float *rewards, const float *values, const 
   const float *tv = truncated ? trunc_value : nullptr;
   return run<TdLambdaOp>(
       pl, N, T, stream,
-      [&](int64_t r0, bool) {
+      [&](int64_t r0) {
         const int64_t o = r0 * T;
         return TdLambdaOp::Args{adv(rewards, o), adv(values, o), adv(bootstrap, r0), adv(tv, o),
                                 adv(terminated, o), adv(truncated, o), adv(returns, o), gamma,
@@ -467,9 +485,9 @@ rlscan_status rlscan_td_lambda(const float *rewards, const float *values, const 
       },
       [&](int64_t r0) {
         const int64_t o = r0 * T;
-        return aligned(adv(rewards, o), 16) && aligned(adv(values, o), 16) &&
-               aligned(adv(returns, o), 16) && aligned(adv(terminated, o), 4) &&
-               aligned(adv(truncated, o), 4);
+        return aligned(adv(rewards, o), 32) && aligned(adv(values, o), 32) &&
+               aligned(adv(returns, o), 32) && aligned(adv(terminated, o), 8) &&
+               aligned(adv(truncated, o), 8);
       });
 }
 
@@ -495,15 +513,15 @@ rlscan_status rlscan_discounted_return(const float *rewards, const float *bootst
   const float *tv = truncated ? trunc_value : nullptr;
   return run<DiscountedOp>(
       pl, N, T, stream,
-      [&](int64_t r0, bool) {
+      [&](int64_t r0) {
         const int64_t o = r0 * T;
         return DiscountedOp::Args{adv(rewards, o), adv(bootstrap, r0), adv(tv, o), adv(terminated, o),
                                   adv(truncated, o), adv(returns, o), gamma};
       },
       [&](int64_t r0) {
         const int64_t o = r0 * T;
-        return aligned(adv(rewards, o), 16) && aligned(adv(returns, o), 16) &&
-               aligned(adv(terminated, o), 4) && aligned(adv(truncated, o), 4);
+        return aligned(adv(rewards, o), 32) && aligned(adv(returns, o), 32) &&
+               aligned(adv(terminated, o), 8) && aligned(adv(truncated, o), 8);
       });
 }
 
@@ -526,15 +544,15 @@ rlscan_status rlscan_elig_trace(const float *inputs, const float *init_trace,
   const Plan pl = make_plan(RLSCAN_EST_ELIG_TRACE, N, T, 1);
   return run<EligOp>(
       pl, N, T, stream,
-      [&](int64_t r0, bool) {
+      [&](int64_t r0) {
         const int64_t o = r0 * T;
         return EligOp::Args{adv(inputs, o), adv(init_trace, r0), adv(terminated, o), adv(truncated, o),
                             adv(traces, o), gamma * lambda};
       },
       [&](int64_t r0) {
         const int64_t o = r0 * T;
-        return aligned(adv(inputs, o), 16) && aligned(adv(traces, o), 16) &&
-               aligned(adv(terminated, o), 4) && aligned(adv(truncated, o), 4);
+        return aligned(adv(inputs, o), 32) && aligned(adv(traces, o), 32) &&
+               aligned(adv(terminated, o), 8) && aligned(adv(truncated, o), 8);
       });
 }
 
@@ -554,14 +572,14 @@ rlscan_status rlscan_episodic_prefix_sum(const int32_t *x, const uint8_t *termin
   const Plan pl = make_plan(RLSCAN_EST_EPISODIC_PREFIX_SUM, N, T, 1);
   return run<PrefixSumOp>(
       pl, N, T, stream,
-      [&](int64_t r0, bool) {
+      [&](int64_t r0) {
         const int64_t o = r0 * T;
         return PrefixSumOp::Args{adv(x, o), adv(terminated, o), adv(truncated, o), adv(out, o)};
       },
       [&](int64_t r0) {
         const int64_t o = r0 * T;
-        return aligned(adv(x, o), 16) && aligned(adv(out, o), 16) && aligned(adv(terminated, o), 4) &&
-               aligned(adv(truncated, o), 4);
+        return aligned(adv(x, o), 32) && aligned(adv(out, o), 32) && aligned(adv(terminated, o), 8) &&
+               aligned(adv(truncated, o), 8);
       });
 }
 
@@ -619,6 +637,12 @@ void rlscan_release_workspaces(void) {
   cudaGetLastError();
 }
 
+rlscan_status rlscan_reserve_workspace(int64_t bytes, rlscan_stream_t stream) {
+  if (bytes < 0) return RLSCAN_ERR_INVALID_ARG;
+  void *ws = nullptr;
+  return get_workspace(stream, std::max<size_t>(size_t(bytes), sizeof(LookbackHeader)), &ws);
+}
+
 int rlscan_abi_version(void) { return RLSCAN_ABI_VERSION; }
 
 rlscan_status rlscan_query_plan(rlscan_estimator est, int64_t N, int64_t T, int64_t A,
@@ -633,7 +657,7 @@ rlscan_status rlscan_query_plan(rlscan_estimator est, int64_t N, int64_t T, int6
   info->chunk_steps = int32_t(pl.L);
   info->lookback = pl.lookback ? 1 : 0;
   info->launches = pl.launches;
-  info->blocks = pl.blocks;
+  info->chunks = pl.chunks;
   info->workspace_bytes = int64_t(pl.ws_bytes);
   return RLSCAN_OK;
 }

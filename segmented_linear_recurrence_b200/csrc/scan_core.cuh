@@ -25,6 +25,17 @@
 
 namespace rlscan {
 
+// Unsigned division by a launch-wide constant d (1 <= d <= 2^30) for
+// numerators below 2^31: q = umulhi(n, m) >> (l - 1) with l = ceil(log2 d) and
+// m = ceil(2^(31+l) / d) (the round-up method of Granlund & Montgomery); the
+// host computes (m, l).  d = 1 is flagged by l = 0.
+struct FastDiv {
+  uint32_t m, l;
+  __device__ __forceinline__ uint32_t div(uint32_t n) const {
+    return l == 0u ? n : (__umulhi(n, m) >> (l - 1u));
+  }
+};
+
 // The affine map x -> b + a * x.
 template <typename V>
 struct Aff {

@@ -132,9 +132,9 @@ def test_valid_call_without_gpu_reports_cuda_error(L):
 def test_query_plan(L):
     p = slr.rlscan_query_plan("gae", 4096, 512)
     assert p["lookback"] == 0 and p["chunk_steps"] % 512 == 0 and p["launches"] == 1
-    assert p["blocks"] == 4096 * 512 // p["chunk_steps"]
+    assert p["chunks"] == 4096 * 512 // p["chunk_steps"]
     p = slr.rlscan_query_plan("vtrace", 256, 16384)
-    assert p["lookback"] == 1 and p["workspace_bytes"] >= 16 * p["blocks"]
+    assert p["lookback"] == 1 and p["workspace_bytes"] >= 16 * p["chunks"]
     p = slr.rlscan_query_plan("retrace", 2048, 512, 18)
     assert p["lookback"] == 0 and p["block_threads"] in (128, 256)
     p = slr.rlscan_query_plan("episodic_prefix_sum", 3, 33)
@@ -142,7 +142,7 @@ def test_query_plan(L):
     # more steps than one launch takes are split by rows
     p = slr.rlscan_query_plan("discounted_return", 1 << 12, 1 << 19)
     assert p["launches"] == 2
-    assert slr.rlscan_query_plan("gae", 0, 5)["blocks"] == 0
+    assert slr.rlscan_query_plan("gae", 0, 5)["chunks"] == 0
 
 
 def test_options_roundtrip(L):
@@ -153,8 +153,9 @@ def test_options_roundtrip(L):
     slr.rlscan_set_option("force_block", 512)
     assert slr.rlscan_query_plan("gae", 64, 32)["block_threads"] == 512
     slr.rlscan_set_option("force_block", 0)
-    with pytest.raises(slr.RlscanError):
-        slr.rlscan_set_option("force_block", 100)
+    for bad in (100, 1024):
+        with pytest.raises(slr.RlscanError):
+            slr.rlscan_set_option("force_block", bad)
     with pytest.raises(slr.RlscanError):
         slr.rlscan_set_option("lookback_timeout_ns", 10)
     slr.rlscan_set_option("force_lookback", 1)

@@ -83,7 +83,8 @@ typedef enum rlscan_status {
   RLSCAN_ERR_TIMEOUT = 4,     /* a thread block gave up waiting for its successor's carry */
   RLSCAN_ERR_NOMEM = 5,       /* workspace allocation failed */
   RLSCAN_ERR_CUDA = 6,        /* another CUDA runtime error (no device, sync failure, ...) */
-  RLSCAN_ERR_CAPTURE = 7      /* workspace would have to grow while the stream is being captured */
+  RLSCAN_ERR_CAPTURE = 7,     /* workspace would have to grow while the stream is being captured */
+  RLSCAN_ERR_TOO_LARGE = 8    /* the problem exceeds rlscan_gae_noalloc's fixed scratch */
 } rlscan_status;
 
 /* ---------------------------------------------------------------------------
@@ -100,6 +101,37 @@ rlscan_status rlscan_gae(const float *rewards, const float *values, const float 
                          const uint8_t *terminated, const uint8_t *truncated,
                          const float *trunc_value, float *advantages, float *returns, int64_t N,
                          int64_t T, float gamma, float lambda, rlscan_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * GAE without any device allocation.  The paper has no counterpart: this is a
+ * deployment variant of rlscan_gae for callers that must not allocate device
+ * memory -- for example code that runs while its stream is being captured
+ * into a CUDA graph (allocation is not a capturable operation), processes in
+ * which another allocator already owns the device's free memory, and
+ * latency-critical loops that cannot afford the device-wide synchronisation
+ * an allocation may cause.  Arguments, layout and results are exactly
+ * rlscan_gae's.
+ *
+ * Scratch.  Rows longer than one thread block's chunk hand carries between
+ * blocks through scratch that here lives in a fixed array compiled into the
+ * library (2 MiB + 16 bytes of device memory on every GPU that loads it, held
+ * until the process exits), instead of a workspace allocated per stream.
+ * - Limit: N * T <= 2^27 steps; larger calls return RLSCAN_ERR_TOO_LARGE and
+ *   launch nothing.
+ * - The first call on a device resolves the array's device address on that
+ *   device (cudaGetSymbolAddress); make that first call before capturing any
+ *   stream into a graph.
+ * - Every call clears the part of the array it uses (one cudaMemsetAsync on
+ *   `stream`) before its kernel, and every call on a device shares the same
+ *   array: calls whose kernels can overlap on the GPU (different streams
+ *   without ordering between them) race on it.  Order them on one stream or
+ *   with events.
+ * ------------------------------------------------------------------------- */
+rlscan_status rlscan_gae_noalloc(const float *rewards, const float *values, const float *bootstrap,
+                                 const uint8_t *terminated, const uint8_t *truncated,
+                                 const float *trunc_value, float *advantages, float *returns,
+                                 int64_t N, int64_t T, float gamma, float lambda,
+                                 rlscan_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * V-trace (Espeholt et al. 2018, IMPALA; named by the pages), with the trace

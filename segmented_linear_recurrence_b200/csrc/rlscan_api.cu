@@ -618,6 +618,7 @@ const char *rlscan_status_string(rlscan_status s) {
     case RLSCAN_ERR_NOMEM: return "RLSCAN_ERR_NOMEM";
     case RLSCAN_ERR_CUDA: return "RLSCAN_ERR_CUDA";
     case RLSCAN_ERR_CAPTURE: return "RLSCAN_ERR_CAPTURE";
+    case RLSCAN_ERR_TOO_LARGE: return "RLSCAN_ERR_TOO_LARGE";
   }
   return "RLSCAN_ERR_UNKNOWN";
 }
@@ -693,3 +694,100 @@ int64_t rlscan_get_option(rlscan_option opt) {
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// rlscan_gae_noalloc: GAE whose look-back scratch is a fixed device array
+// ===========================================================================
+// For callers that must not allocate device memory (graph capture, foreign
+// allocators, latency-critical loops): the carry hand-off between thread
+// blocks uses this file-scope array instead of a per-stream workspace.  Host
+// code cannot use the array's name as a device address; its address is
+// resolved once per device with cudaGetSymbolAddress.
+namespace {
+
+constexpr int64_t kNoAllocMaxSteps = int64_t(1) << 27;
+// Header plus one descriptor per chunk of the smallest chunk size (1024 steps).
+constexpr size_t kNoAllocScratchBytes =
+    sizeof(LookbackHeader) + sizeof(LookbackDesc) * size_t(kNoAllocMaxSteps / 1024);
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device (set up on the
+// first call per device, with that device current).
+rlscan_status noalloc_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) {
+    cudaGetLastError();
+    return RLSCAN_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return RLSCAN_ERR_CUDA;
+    }
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = g_noalloc_addr[dev];
+  return RLSCAN_OK;
+}
+
+}  // namespace
+
+extern "C" rlscan_status rlscan_gae_noalloc(const float *rewards, const float *values, const float *bootstrap,
+                                            const uint8_t *terminated, const uint8_t *truncated,
+                                            const float *trunc_value, float *advantages, float *returns,
+                                            int64_t N, int64_t T, float gamma, float lambda,
+                                            rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  if (N * T > kNoAllocMaxSteps) return RLSCAN_ERR_TOO_LARGE;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(rewards), c.need(values), c.need(bootstrap), c.need(advantages);
+  if (truncated) c.need(trunc_value);
+  c.finite(gamma), c.finite(lambda);
+  c.input(rewards, nt * 4, 4), c.input(values, nt * 4, 4), c.input(bootstrap, size_t(N) * 4, 4);
+  c.input(terminated, nt, 1), c.input(truncated, nt, 1);
+  if (truncated) c.input(trunc_value, nt * 4, 4);
+  c.output(advantages, nt * 4, 4), c.output(returns, nt * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+
+  const Plan pl = make_plan(RLSCAN_EST_GAE, N, T, 1);  // N * T <= 2^27: a single launch
+  ScanGeom g{};
+  g.total = uint32_t(nt);
+  g.T = uint32_t(T);
+  g.nchunks = uint32_t((nt + pl.L - 1) / pl.L);
+  g.vec = (g_force_scalar.load() == 0 && aligned(rewards, 32) && aligned(values, 32) && aligned(advantages, 32) &&
+           aligned(returns, 32) && aligned(terminated, 8) && aligned(truncated, 8))
+              ? 1u
+              : 0u;
+  fast_div_params(uint32_t(T), g.div_m, g.div_l);
+  g.lb.timeout_ns = uint64_t(std::max<int64_t>(1000, g_timeout_ns.load()));
+  g.lb.starve = 0u;
+  if (pl.lookback) {
+    void *scratch = nullptr;
+    const rlscan_status st = noalloc_scratch(&scratch);
+    if (st != RLSCAN_OK) return st;
+    // Start from a clean header and clean descriptors for this call's chunks.
+    const size_t used = sizeof(LookbackHeader) + size_t(g.nchunks) * sizeof(LookbackDesc);
+    if (cudaMemsetAsync(scratch, 0, used, stream) != cudaSuccess) {
+      cudaGetLastError();
+      return RLSCAN_ERR_CUDA;
+    }
+    g.lb.hdr = static_cast<LookbackHeader *>(scratch);
+    g.lb.desc = reinterpret_cast<LookbackDesc *>(static_cast<LookbackHeader *>(scratch) + 1);
+  }
+  const float *tv = truncated ? trunc_value : nullptr;
+  const GaeOp::Args a{rewards, values, bootstrap, tv, terminated, truncated, advantages, returns, gamma,
+                      gamma * lambda};
+  const cudaError_t e = launch_block<GaeOp>(a, g, pl.block, pl.lookback, stream);
+  return e == cudaSuccess ? RLSCAN_OK : RLSCAN_ERR_LAUNCH;
+}

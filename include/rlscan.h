@@ -267,12 +267,16 @@ rlscan_status rlscan_query_plan(rlscan_estimator estimator, int64_t N, int64_t T
 typedef enum rlscan_option {
   RLSCAN_OPT_LOOKBACK_TIMEOUT_NS = 1, /* carry wait limit per block, default 1e9 (1 s) */
   RLSCAN_OPT_FORCE_LOOKBACK = 2,      /* 1: chain carries even where blocks hold whole rows */
-  RLSCAN_OPT_FORCE_BLOCK = 3,         /* 0: auto; else threads per block (128, 256, 512;
-                                         Retrace takes 128 or 256 and ignores other values) */
+  RLSCAN_OPT_FORCE_BLOCK = 3,         /* 0: auto; else threads per block (a multiple of 64
+                                         from 128 to 512; Retrace takes 128 or 256 and
+                                         ignores other values) */
   RLSCAN_OPT_FORCE_SCALAR = 4,        /* 1: take the scalar (unvectorised) load path */
   RLSCAN_OPT_CHECK_POINTERS = 5,      /* default 1: reject host memory the device cannot read */
-  RLSCAN_OPT_TEST_STARVE_LOOKBACK = 6 /* test only, 1: the first block never publishes its
-                                         carry, so its predecessors time out */
+  RLSCAN_OPT_TEST_STARVE_LOOKBACK = 6, /* test only, 1: the first block never publishes its
+                                          carry, so its predecessors time out */
+  RLSCAN_OPT_PDL = 7                   /* default 1: programmatic dependent launch, so a kernel
+                                          can be scheduled while the previous kernel on the
+                                          stream drains (it waits for it before any access) */
 } rlscan_option;
 
 rlscan_status rlscan_set_option(rlscan_option option, int64_t value);

@@ -34,7 +34,7 @@ STATUS = {0: "RLSCAN_OK", 1: "RLSCAN_ERR_INVALID_ARG", 2: "RLSCAN_ERR_OVERLAP",
           3: "RLSCAN_ERR_LAUNCH", 4: "RLSCAN_ERR_TIMEOUT", 5: "RLSCAN_ERR_NOMEM",
           6: "RLSCAN_ERR_CUDA", 7: "RLSCAN_ERR_CAPTURE", 8: "RLSCAN_ERR_TOO_LARGE"}
 OPTIONS = {"lookback_timeout_ns": 1, "force_lookback": 2, "force_block": 3, "force_scalar": 4,
-           "check_pointers": 5, "test_starve_lookback": 6}
+           "check_pointers": 5, "test_starve_lookback": 6, "pdl": 7}
 ESTIMATOR_IDS = {"gae": 0, "vtrace": 1, "retrace": 2, "td_lambda": 3, "discounted_return": 4,
                  "elig_trace": 5, "episodic_prefix_sum": 6}
 

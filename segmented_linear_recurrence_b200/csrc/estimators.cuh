@@ -39,13 +39,14 @@ constexpr int kTile = 8;  // consecutive steps per thread
 
 // Geometry of one thread's tile.
 struct Tile {
-  uint32_t i0;     // first step (flat, launch-local)
-  int nvalid;      // steps of the tile inside the launch (0..8)
-  uint32_t valid;  // bit k: step k exists
+  uint32_t i0;     // first step (flat, launch-local; a multiple of 8)
+  int nvalid;      // steps of the tile inside the launch (0..8): these may be loaded
+  uint32_t valid;  // bit k: step k belongs to this block (scanned and stored)
   uint32_t n0, t0; // row and time of step i0
   uint32_t edge;   // bit k: step k is on its row's dependency edge
                    //   (backward: t = T-1, forward: t = 0)
-  bool fast;       // 256-bit (flags: 64-bit) accesses allowed
+  bool fast;       // 256-bit (flags: 64-bit) loads allowed
+  bool full;       // ... and all 8 steps are the block's: 256-bit stores
   bool few_rows;   // T >= 8: at most one row edge in the tile
 };
 
@@ -96,26 +97,26 @@ __device__ __forceinline__ uint32_t ld8_flags(const uint8_t *p, const Tile &tl) 
 }
 
 __device__ __forceinline__ void st8(float *p, const Tile &tl, const float (&v)[8]) {
-  if (tl.fast) {
+  if (tl.full) {
     asm volatile("st.global.cs.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p + tl.i0), "f"(v[0]), "f"(v[1]),
                  "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
                  : "memory");
   } else {
 #pragma unroll
     for (int k = 0; k < 8; ++k)
-      if (k < tl.nvalid) p[tl.i0 + k] = v[k];
+      if ((tl.valid >> k) & 1u) p[tl.i0 + k] = v[k];
   }
 }
 
 __device__ __forceinline__ void st8(int32_t *p, const Tile &tl, const uint32_t (&v)[8]) {
-  if (tl.fast) {
+  if (tl.full) {
     asm volatile("st.global.cs.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p + tl.i0), "r"(v[0]), "r"(v[1]),
                  "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
                  : "memory");
   } else {
 #pragma unroll
     for (int k = 0; k < 8; ++k)
-      if (k < tl.nvalid) p[tl.i0 + k] = int32_t(v[k]);
+      if ((tl.valid >> k) & 1u) p[tl.i0 + k] = int32_t(v[k]);
   }
 }
 
@@ -136,6 +137,9 @@ __device__ __forceinline__ void boundary_values(const float *tv, const float *bo
   const uint32_t tr = trunc & ~term & tl.valid;
   const uint32_t ed = tl.edge & ~term & ~trunc;
 #pragma unroll
+  for (int k = 0; k < 8; ++k) sv[k] = 0.0f;
+  if (!__any_sync(0xffffffffu, (tr | ed) != 0u)) return;  // most warps: nothing to fetch
+#pragma unroll
   for (int k = 0; k < 8; ++k) {
     float s = 0.0f;
     if ((tr >> k) & 1u)
@@ -151,6 +155,7 @@ __device__ __forceinline__ void boundary_values(const float *tv, const float *bo
 // b = r + gamma nv - v.  Outputs advantages = x, returns = x + v.
 // ---------------------------------------------------------------------------
 struct GaeOp {
+  static constexpr int kRegs = 40, kRegsLookback = 48;  // registers per thread (see scan_kernel.cuh)
   using V = float;
   static constexpr bool kBackward = true;
   struct Args {
@@ -206,6 +211,7 @@ struct GaeOp {
 // inside an episode, b = r + gamma nv at a boundary.  Output x.
 // ---------------------------------------------------------------------------
 struct TdLambdaOp {
+  static constexpr int kRegs = 40, kRegsLookback = 48;  // registers per thread (see scan_kernel.cuh)
   using V = float;
   static constexpr bool kBackward = true;
   struct Args {
@@ -253,6 +259,7 @@ struct TdLambdaOp {
 // bootstrap may be NULL (zero at the window end).  Output x.
 // ---------------------------------------------------------------------------
 struct DiscountedOp {
+  static constexpr int kRegs = 32, kRegsLookback = 48;  // registers per thread (see scan_kernel.cuh)
   using V = float;
   static constexpr bool kBackward = true;
   struct Args {
@@ -300,6 +307,7 @@ struct DiscountedOp {
 // episode (vs_{t+1} = v_{t+1} + x_{t+1}), rho (r + gamma nv - v) at a boundary.
 // ---------------------------------------------------------------------------
 struct VtraceOp {
+  static constexpr int kRegs = 48, kRegsLookback = 56;  // registers per thread (see scan_kernel.cuh)
   using V = float;
   static constexpr bool kBackward = true;
   struct Args {
@@ -362,6 +370,7 @@ struct VtraceOp {
 // b = g + gamma lambda init[n], a = 0.  Output x.
 // ---------------------------------------------------------------------------
 struct EligOp {
+  static constexpr int kRegs = 32, kRegsLookback = 48;  // registers per thread (see scan_kernel.cuh)
   using V = float;
   static constexpr bool kBackward = false;
   struct Args {
@@ -409,6 +418,7 @@ struct EligOp {
 // a = 0 at a row start or after a done step, else 1; b = x.
 // ---------------------------------------------------------------------------
 struct PrefixSumOp {
+  static constexpr int kRegs = 32, kRegsLookback = 48;  // registers per thread (see scan_kernel.cuh)
   using V = uint32_t;
   static constexpr bool kBackward = false;
   struct Args {

@@ -296,19 +296,14 @@ __global__ void __launch_bounds__(BLOCK) retrace_kernel(const RetraceOp::Args p,
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const FastDiv fd{g.div_m, g.div_l};
+  grid_dependency_wait();
   uint32_t chunk = blockIdx.x, ticket = 0, epoch = 0;
   if constexpr (LB) {
-    if (tid == 0) {
-      s_ticket = atomicInc(&g.lb.hdr->ticket, g.fetch_wrap);
-      s_epoch = *reinterpret_cast<volatile uint32_t *>(&g.lb.hdr->epoch);
-    }
+    if (tid == 0 && !draw_ticket(g.lb.hdr, g.nchunks, s_ticket, s_epoch)) record_status(kDevStatusTimeout);
     __syncthreads();
     ticket = s_ticket;
     epoch = s_epoch;
-    if (ticket >= g.nchunks) {  // counter left inconsistent by an aborted launch
-      if (tid == 0) record_status(kDevStatusTimeout);
-      return;
-    }
+    if (ticket >= g.nchunks) return;  // counter left inconsistent by an aborted launch
     chunk = g.nchunks - 1u - ticket;
   }
   const uint32_t cbase = chunk * L;
@@ -323,6 +318,7 @@ __global__ void __launch_bounds__(BLOCK) retrace_kernel(const RetraceOp::Args p,
   }
   Item it[4];
   Op::load(p, i0, nvalid, g.vec != 0u, it);
+  grid_dependents_launch();
   Nbr nb[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) nb[k] = Op::nbr_smem(dyn_smem, L, 4u * uint32_t(tid) + k + 1u);
@@ -356,12 +352,9 @@ __global__ void __launch_bounds__(BLOCK) retrace_kernel(const RetraceOp::Args p,
     if constexpr (LB) {
       const V ca = __shfl_sync(0xffffffffu, winc.a, 0);
       const V cb = __shfl_sync(0xffffffffu, winc.b, 0);
-      if (lane == 0) {
-        const bool edge_closed = (min(cbase + L, g.total) % g.T) == 0u;
-        carry = decoupled_lookback<true, V>(g.lb, chunk, g.nchunks, epoch, ticket, Aff<V>{ca, cb},
-                                            edge_closed);
-      }
-      carry = __shfl_sync(0xffffffffu, carry, 0);
+      const bool edge_closed = (min(cbase + L, g.total) % g.T) == 0u;
+      carry = decoupled_lookback<true, V>(g.lb, chunk, g.nchunks, epoch, ticket, Aff<V>{ca, cb}, edge_closed,
+                                          lane);
     }
     if (lane < W) s_wcarry[lane] = apply(wexc, carry);
   }
@@ -376,13 +369,6 @@ __global__ void __launch_bounds__(BLOCK) retrace_kernel(const RetraceOp::Args p,
     xs[k] = x;
   }
   Op::emit(p, i0, nvalid, g.vec != 0u, it, xs, xd, aux);
-
-  if constexpr (LB) {
-    if (tid == 0) {
-      __threadfence();
-      if (atomicInc(&g.lb.hdr->done, g.nchunks - 1u) == g.nchunks - 1u) atomicAdd(&g.lb.hdr->epoch, 1u);
-    }
-  }
 }
 
 }  // namespace rlscan

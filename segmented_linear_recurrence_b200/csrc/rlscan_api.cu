@@ -34,6 +34,25 @@ std::atomic<int64_t> g_force_block{0};
 std::atomic<int64_t> g_force_scalar{0};
 std::atomic<int64_t> g_check_pointers{1};
 std::atomic<int64_t> g_starve{0};
+std::atomic<int64_t> g_pdl{1};
+
+// Launch with programmatic stream serialization (when enabled), so the grid
+// can be scheduled while the previous kernel on the stream drains; the kernels
+// wait for that kernel before touching memory.
+template <class Kernel, class... Args>
+cudaError_t launch(Kernel kern, uint32_t grid, int block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g_pdl.load() != 0 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 
 constexpr int64_t kMaxStepsPerLaunch = int64_t(1) << 30;
 constexpr int64_t kMaxRowSteps = int64_t(1) << 30;
@@ -183,7 +202,8 @@ bool aligned(const void *p, uintptr_t a) { return p == nullptr || reinterpret_ca
 // ---------------------------------------------------------------------------
 struct Plan {
   int block = 256;
-  uint32_t L = 2048;        // steps per chunk
+  uint32_t L = 2048;        // steps per chunk (look-back plan); rows plan: steps per block
+  int64_t rows_per_block = 0;  // rows plan: whole rows per block
   bool lookback = false;
   int64_t rows_per_launch = 0;
   int launches = 0;
@@ -195,34 +215,66 @@ struct Plan {
   size_t smem = 0;
 };
 
-bool valid_block(int64_t b) { return b == 128 || b == 256 || b == 512; }
+// Thread blocks (chunks) of one launch over `rows` rows.
+uint32_t blocks_in_launch(const Plan &pl, int64_t rows, int64_t T) {
+  return pl.rows_per_block > 0 ? uint32_t((rows + pl.rows_per_block - 1) / pl.rows_per_block)
+                               : uint32_t((rows * T + pl.L - 1) / pl.L);
+}
+
+// Threads per block of the scan kernels: multiples of 64 from 128 to 512, so
+// that whole rows can fill a block closely.
+constexpr int kBlocks[] = {128, 192, 256, 320, 384, 448, 512};
+bool valid_block(int64_t b) { return b >= 128 && b <= 512 && b % 64 == 0; }
+
+// Rows plan: the most whole rows of T steps a block of `block` threads can
+// own, whatever the alignment of its first step (0 if one row does not fit).
+// k rows span k T steps, whose 8-step tiles number k T / 8 when k T is a
+// multiple of 8 (every block then starts aligned) and at most
+// (k T + 14) / 8 otherwise.
+int64_t rows_per_block(int64_t T, int block) {
+  auto tiles = [T](int64_t k) { return (k * T) % kTile == 0 ? k * T / kTile : (k * T + 2 * kTile - 2) / kTile; };
+  int64_t k = int64_t(kTile) * block / T;
+  while (k > 0 && tiles(k) > block) --k;
+  return k;
+}
 
 Plan make_plan(rlscan_estimator est, int64_t N, int64_t T, int64_t A) {
   Plan pl;
   const int64_t fb = g_force_block.load();
+  const bool force_lb = g_force_lookback.load() != 0;
   if (est == RLSCAN_EST_RETRACE) {
     pl.block = (fb == 128 || fb == 256) ? int(fb) : 128;
     pl.L = 4u * uint32_t(pl.block);
+    pl.lookback = force_lb || (int64_t(pl.L) % T) != 0;
   } else {
-    if (valid_block(fb)) {
-      pl.block = int(fb);
-    } else {
-      pl.block = 0;
-      for (int b : {128, 256, 512})
-        if ((int64_t(kTile) * b) % T == 0) {
-          pl.block = b;
-          break;
-        }
-      if (pl.block == 0) pl.block = 256;
+    // Rows plan where a row fits a block: the block size whose threads the
+    // rows fill best (the smaller one on a tie); else the look-back plan.
+    int64_t best_k = 0;
+    pl.block = 256;
+    double best_fill = 0.0;
+    for (int b : kBlocks) {
+      if (valid_block(fb) && b != fb) continue;
+      const int64_t k = rows_per_block(T, b);
+      const double fill = double(k * T) / double(int64_t(kTile) * b);
+      if (k > 0 && fill > best_fill + 1e-9) {
+        best_fill = fill;
+        best_k = k;
+        pl.block = b;
+      }
     }
-    pl.L = uint32_t(kTile) * uint32_t(pl.block);
+    if (valid_block(fb)) pl.block = int(fb);
+    pl.lookback = force_lb || best_k == 0;
+    if (pl.lookback) {
+      pl.L = uint32_t(kTile) * uint32_t(pl.block);
+    } else {
+      pl.rows_per_block = best_k;
+      pl.L = uint32_t(best_k * T);
+    }
   }
-  pl.lookback = g_force_lookback.load() != 0 || (int64_t(pl.L) % T) != 0;
   pl.rows_per_launch = std::max<int64_t>(1, kMaxStepsPerLaunch / T);
   pl.launches = int((N + pl.rows_per_launch - 1) / pl.rows_per_launch);
   for (int64_t r0 = 0; r0 < N; r0 += pl.rows_per_launch) {
-    const int64_t rows = std::min(pl.rows_per_launch, N - r0);
-    const uint32_t nch = uint32_t((rows * T + pl.L - 1) / pl.L);
+    const uint32_t nch = blocks_in_launch(pl, std::min(pl.rows_per_launch, N - r0), T);
     pl.chunks += nch;
     pl.max_chunks = std::max(pl.max_chunks, nch);
   }
@@ -256,17 +308,23 @@ void fast_div_params(uint32_t d, uint32_t &m, uint32_t &l) {
 
 template <class Op, int BLOCK, bool LB>
 cudaError_t launch_scan(const typename Op::Args &a, ScanGeom g, cudaStream_t s) {
-  g.fetch_wrap = g.nchunks - 1u;  // one ticket per block
-  scan_kernel<Op, BLOCK, LB><<<g.nchunks, BLOCK, 0, s>>>(a, g);
-  return cudaGetLastError();
+  const cudaError_t e = launch(scan_kernel<Op, BLOCK, LB>, g.nchunks, BLOCK, 0, s, a, g);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <class Op>
 cudaError_t launch_block(const typename Op::Args &a, const ScanGeom &g, int block, bool lb, cudaStream_t s) {
   switch (block) {
-    case 128: return lb ? launch_scan<Op, 128, true>(a, g, s) : launch_scan<Op, 128, false>(a, g, s);
-    case 256: return lb ? launch_scan<Op, 256, true>(a, g, s) : launch_scan<Op, 256, false>(a, g, s);
-    case 512: return lb ? launch_scan<Op, 512, true>(a, g, s) : launch_scan<Op, 512, false>(a, g, s);
+#define RLSCAN_BLOCK_CASE(B) \
+  case B: return lb ? launch_scan<Op, B, true>(a, g, s) : launch_scan<Op, B, false>(a, g, s);
+    RLSCAN_BLOCK_CASE(128)
+    RLSCAN_BLOCK_CASE(192)
+    RLSCAN_BLOCK_CASE(256)
+    RLSCAN_BLOCK_CASE(320)
+    RLSCAN_BLOCK_CASE(384)
+    RLSCAN_BLOCK_CASE(448)
+    RLSCAN_BLOCK_CASE(512)
+#undef RLSCAN_BLOCK_CASE
     default: return cudaErrorInvalidValue;
   }
 }
@@ -278,9 +336,8 @@ cudaError_t launch_retrace(const RetraceOp::Args &a, ScanGeom g, size_t smem, cu
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
   }
-  g.fetch_wrap = g.nchunks - 1u;
-  kern<<<g.nchunks, BLOCK, smem, s>>>(a, g);
-  return cudaGetLastError();
+  const cudaError_t e = launch(kern, g.nchunks, BLOCK, smem, s, a, g);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_retrace_block(const RetraceOp::Args &a, const ScanGeom &g, int block, bool lb, size_t smem,
@@ -306,7 +363,8 @@ rlscan_status run(const Plan &pl, int64_t N, int64_t T, rlscan_stream_t stream, 
     ScanGeom g{};
     g.total = uint32_t(rows * T);
     g.T = uint32_t(T);
-    g.nchunks = uint32_t((rows * T + pl.L - 1) / pl.L);
+    g.nchunks = blocks_in_launch(pl, rows, T);
+    g.span = pl.L;
     const bool vec = g_force_scalar.load() == 0 && slice_vec(r0);
     g.vec = vec ? 1u : 0u;
     fast_div_params(uint32_t(T), g.div_m, g.div_l);
@@ -677,6 +735,7 @@ rlscan_status rlscan_set_option(rlscan_option opt, int64_t v) {
     case RLSCAN_OPT_FORCE_SCALAR: g_force_scalar = v ? 1 : 0; return RLSCAN_OK;
     case RLSCAN_OPT_CHECK_POINTERS: g_check_pointers = v ? 1 : 0; return RLSCAN_OK;
     case RLSCAN_OPT_TEST_STARVE_LOOKBACK: g_starve = v ? 1 : 0; return RLSCAN_OK;
+    case RLSCAN_OPT_PDL: g_pdl = v ? 1 : 0; return RLSCAN_OK;
   }
   return RLSCAN_ERR_INVALID_ARG;
 }
@@ -689,6 +748,7 @@ int64_t rlscan_get_option(rlscan_option opt) {
     case RLSCAN_OPT_FORCE_SCALAR: return g_force_scalar.load();
     case RLSCAN_OPT_CHECK_POINTERS: return g_check_pointers.load();
     case RLSCAN_OPT_TEST_STARVE_LOOKBACK: return g_starve.load();
+    case RLSCAN_OPT_PDL: return g_pdl.load();
   }
   return -1;
 }
@@ -764,7 +824,8 @@ extern "C" rlscan_status rlscan_gae_noalloc(const float *rewards, const float *v
   ScanGeom g{};
   g.total = uint32_t(nt);
   g.T = uint32_t(T);
-  g.nchunks = uint32_t((nt + pl.L - 1) / pl.L);
+  g.nchunks = blocks_in_launch(pl, N, T);
+  g.span = pl.L;
   g.vec = (g_force_scalar.load() == 0 && aligned(rewards, 32) && aligned(values, 32) && aligned(advantages, 32) &&
            aligned(returns, 32) && aligned(terminated, 8) && aligned(truncated, 8))
               ? 1u

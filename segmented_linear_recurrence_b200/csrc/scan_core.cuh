@@ -36,6 +36,13 @@ struct FastDiv {
   }
 };
 
+// Programmatic dependent launch (sm_90+): both are no-ops when the grid was
+// launched without the programmatic-serialization attribute.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // The affine map x -> b + a * x.
 template <typename V>
 struct Aff {
@@ -109,47 +116,60 @@ __device__ __forceinline__ void record_status(uint32_t code) {
 // ---------------------------------------------------------------------------
 // Decoupled look-back workspace.
 // ---------------------------------------------------------------------------
-// Per launch: a ticket counter hands out chunk indices in dependency order (so
-// every chunk a block waits on belongs to a block that is already running),
-// a done counter lets the last block reset both counters and advance the
-// epoch, and every descriptor's flag carries the epoch of the launch that
-// wrote it, so descriptors left over from earlier launches are never read as
-// current and the workspace never needs clearing between launches.
+// Per launch: one 64-bit counter, (epoch << 32) | next ticket, hands out
+// chunk indices in dependency order (so every chunk a block waits on belongs
+// to a block that is already running) together with the launch's epoch, in
+// a single atomic.  The block that draws the launch's last ticket moves the
+// counter on to (epoch + 1, 0); no other block touches it afterwards, and
+// stream order keeps the next launch from drawing before this one has ended.
+// Every descriptor's flag carries the epoch of the launch that wrote it, so
+// descriptors left over from earlier launches are never read as current and
+// the workspace never needs clearing between launches.  A launch that ends
+// early (a dead context) leaves the counter inconsistent; the next launch
+// reports it as a timeout, and releasing the workspaces clears it.
 struct LookbackHeader {
-  uint32_t ticket;
-  uint32_t done;
-  uint32_t epoch;
-  uint32_t pad;
+  unsigned long long counter;
+  unsigned long long pad;
 };
 
-// flag = (epoch << 2) | state.  State 1: the chunk's aggregate (a, b) is
-// published.  State 2: its outgoing value x is published -- the scan value at
-// the step its dependent neighbour reads as carry (backward: the chunk's
-// first step; forward: its last step).
+// Draws this block's ticket and the launch's epoch.  False if the counter was
+// left inconsistent (ticket out of range).
+__device__ __forceinline__ bool draw_ticket(LookbackHeader *h, uint32_t nchunks, uint32_t &ticket,
+                                            uint32_t &epoch) {
+  const unsigned long long old = atomicAdd(&h->counter, 1ull);
+  ticket = uint32_t(old);
+  epoch = uint32_t(old >> 32);
+  if (ticket == nchunks - 1u) atomicAdd(&h->counter, (1ull << 32) - nchunks);
+  return ticket < nchunks;
+}
+
+// A chunk's descriptor is two 64-bit words, each (flag << 32) | value with
+// flag = (epoch << 2) | state, written and read as single-copy-atomic 64-bit
+// accesses.  Every word validates itself, so no fence orders one word against
+// another:
+//   word 0 = (A, a): the chunk's aggregate's a;  word 1 = (A, b): its b;
+//   word 0 = (P, x): its outgoing value x, the scan value at the step its
+//            dependent neighbour reads as carry (backward: the chunk's first
+//            step; forward: its last step).  Replaces (A, a) when known.
+// A reader that sees (P, x) in word 0 is done; one that sees (A, a) needs
+// (A, b) in word 1 too, and otherwise polls again.
 struct LookbackDesc {
-  uint32_t flag;
-  uint32_t a;
-  uint32_t b;
-  uint32_t x;
+  unsigned long long w[2];
 };
 
 enum : uint32_t { kDescAggregate = 1, kDescInclusive = 2 };
 
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
+__device__ __forceinline__ unsigned long long desc_word(uint32_t flag, uint32_t value) {
+  return (static_cast<unsigned long long>(flag) << 32) | value;
 }
-__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t *p) {
-  uint32_t v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
-__device__ __forceinline__ void st_release_u32(uint32_t *p, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ void st_relaxed_u32(uint32_t *p, uint32_t v) {
-  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+// Both words of a descriptor in one access; each 64-bit element is
+// single-copy atomic on its own, which is all the protocol needs.
+__device__ __forceinline__ void ld_relaxed_desc(const LookbackDesc *p, unsigned long long &w0,
+                                                unsigned long long &w1) {
+  asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(w0), "=l"(w1) : "l"(p) : "memory");
 }
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
@@ -177,81 +197,111 @@ struct LookbackCtl {
   uint32_t starve;  // test only: the block holding ticket 0 never publishes
 };
 
-// Run by one thread per block.  Publishes the chunk's aggregate (or its final
-// value at once if the aggregate already cuts the dependency), finds the
-// carry entering the chunk's dependency edge by walking successors (backward)
-// or predecessors (forward), then publishes the chunk's final value.
+// Run by all 32 lanes of one warp per block.  Lane 0 publishes the chunk's
+// aggregate (or its final value at once if the aggregate already cuts the
+// dependency).  The warp then finds the carry entering the chunk's
+// dependency edge by polling the descriptors of the next 32 chunks in
+// dependency order at once (successors backward, predecessors forward): the
+// nearest one that is final -- published value, an aggregate that cuts, or
+// the end of the array -- ends the walk as soon as it and every descriptor
+// before it are ready, and the aggregates before it are composed with one
+// warp scan.  One window normally suffices; otherwise the window slides by
+// 32.  Lane 0 finally publishes the chunk's value.
 //
 // `edge_closed`: the chunk's dependency edge is a row boundary, so its
 // elements need no carry.  Every wait is bounded by `timeout_ns` of global
 // time (and an iteration cap as a second bound); on expiry the block records
-// RLSCAN timeout status, uses the partial carry, and still publishes so no
-// other block waits on it.
+// the timeout status, uses the partial carry, and still publishes so no other
+// block waits on it.
 template <bool BACKWARD, typename V>
-__device__ V decoupled_lookback(const LookbackCtl &ctl, uint32_t chunk, uint32_t nchunks,
-                                uint32_t epoch, uint32_t ticket, Aff<V> agg, bool edge_closed) {
+__device__ V decoupled_lookback(const LookbackCtl &ctl, uint32_t chunk, uint32_t nchunks, uint32_t epoch,
+                                uint32_t ticket, Aff<V> agg, bool edge_closed, int lane) {
   const uint32_t tag = epoch << 2;
   const bool silent = ctl.starve && ticket == 0;
   LookbackDesc *mine = ctl.desc + chunk;
   const bool self_cut = cuts(agg);
-  if (!silent) {
+  if (lane == 0 && !silent) {
     if (self_cut) {
-      st_relaxed_u32(&mine->x, to_bits(agg.b));
-      st_release_u32(&mine->flag, tag | kDescInclusive);
+      st_relaxed_u64(&mine->w[0], desc_word(tag | kDescInclusive, to_bits(agg.b)));
     } else {
-      st_relaxed_u32(&mine->a, to_bits(agg.a));
-      st_relaxed_u32(&mine->b, to_bits(agg.b));
-      st_release_u32(&mine->flag, tag | kDescAggregate);
+      st_relaxed_u64(&mine->w[1], desc_word(tag | kDescAggregate, to_bits(agg.b)));
+      st_relaxed_u64(&mine->w[0], desc_word(tag | kDescAggregate, to_bits(agg.a)));
     }
   }
   V carry = V(0);
   if (!edge_closed) {
     Aff<V> acc = aff_identity<V>();
-    int64_t j = BACKWARD ? int64_t(chunk) + 1 : int64_t(chunk) - 1;
-    bool resolved = false;
-    const uint64_t t0 = global_timer_ns();
-    const uint64_t max_iters = 64 + ctl.timeout_ns / 64;
-    while (!resolved && j >= 0 && j < int64_t(nchunks)) {
-      const LookbackDesc *d = ctl.desc + j;
-      uint32_t f = 0;
-      uint32_t sleep_ns = 32;
-      uint64_t iters = 0;
+    // 32-bit bookkeeping keeps the walk light in registers: chunk indices fit
+    // (nchunks < 2^31), and the timer's low word measures waits up to 2^31 ns.
+    int32_t base = BACKWARD ? int32_t(chunk) + 1 : int32_t(chunk) - 1;
+    const uint32_t t0 = uint32_t(global_timer_ns());
+    const uint32_t limit_ns = uint32_t(min(ctl.timeout_ns, uint64_t(1) << 31));
+    const uint32_t max_polls = 64u + limit_ns / 32u;
+    uint32_t polls = 0;
+    for (;;) {
+      // Lane i looks at the i-th predecessor of the window.  Each lane polls
+      // its descriptor only until it is ready; the window is usable as soon
+      // as every lane up to the nearest final one is ready, so a far lane
+      // never holds up the walk.  Past the array end nothing enters.
+      const int32_t j = base + (BACKWARD ? lane : -lane);
+      const bool in_range = j >= 0 && uint32_t(j) < nchunks;
+      const LookbackDesc *d = ctl.desc + (in_range ? j : 0);
+      bool ready = !in_range, final_here = !in_range;
+      Aff<V> e = aff_identity<V>();
+      V xval = V(0);
+      uint32_t sleep_ns = 0;
       bool timed_out = false;
+      uint32_t fmask, lead;
       for (;;) {
-        f = ld_acquire_u32(&d->flag);
-        if ((f & ~3u) == tag && (f & 3u) != 0u) break;
-        if (++iters > max_iters || global_timer_ns() - t0 > ctl.timeout_ns) {
+        if (!ready) {
+          unsigned long long w0, w1;
+          ld_relaxed_desc(d, w0, w1);
+          const uint32_t f0 = uint32_t(w0 >> 32);
+          if (f0 == (tag | kDescInclusive)) {
+            ready = final_here = true;
+            xval = from_bits<V>(uint32_t(w0));
+          } else if (f0 == (tag | kDescAggregate) && uint32_t(w1 >> 32) == (tag | kDescAggregate)) {
+            ready = true;
+            e = Aff<V>{from_bits<V>(uint32_t(w0)), from_bits<V>(uint32_t(w1))};
+            if (cuts(e)) {  // an aggregate that cuts carries its own value
+              final_here = true;
+              xval = e.b;
+            }
+          }
+        }
+        const uint32_t rmask = __ballot_sync(0xffffffffu, ready);
+        fmask = __ballot_sync(0xffffffffu, final_here);
+        lead = rmask == 0xffffffffu ? 32u : uint32_t(__ffs(~rmask) - 1);  // ready lanes 0..lead-1
+        const uint32_t first = fmask ? uint32_t(__ffs(fmask) - 1) : 32u;
+        if (first < lead || lead == 32u) break;
+        // lanes may read the timer a tick apart: decide for the whole warp
+        const bool expired = ++polls > max_polls || uint32_t(global_timer_ns()) - t0 > limit_ns;
+        if (__any_sync(0xffffffffu, expired)) {
           timed_out = true;
           break;
         }
-        __nanosleep(sleep_ns);
-        if (sleep_ns < 1024) sleep_ns <<= 1;
+        if (sleep_ns) __nanosleep(sleep_ns);
+        sleep_ns = sleep_ns ? min(sleep_ns * 2u, 256u) : 16u;
       }
       if (timed_out) {
-        record_status(kDevStatusTimeout);
+        if (lane == 0) record_status(kDevStatusTimeout);
         carry = acc.b;
-        resolved = true;
         break;
       }
-      if ((f & 3u) == kDescInclusive) {
-        carry = apply(acc, from_bits<V>(ld_relaxed_u32(&d->x)));
-        resolved = true;
-      } else {
-        Aff<V> pa{from_bits<V>(ld_relaxed_u32(&d->a)), from_bits<V>(ld_relaxed_u32(&d->b))};
-        acc = compose(acc, pa);
-        if (cuts(acc)) {
-          carry = acc.b;
-          resolved = true;
-        }
-        j += BACKWARD ? 1 : -1;
+      const int first = fmask ? __ffs(fmask) - 1 : 32;
+      // lanes 0..first-1 in dependency order, the nearest outermost
+      const Aff<V> win = warp_inclusive_scan<true>(lane < first ? e : aff_identity<V>(), lane);
+      const V wa = __shfl_sync(0xffffffffu, win.a, 0);
+      const V wb = __shfl_sync(0xffffffffu, win.b, 0);
+      acc = compose(acc, Aff<V>{wa, wb});
+      if (first < 32) {
+        carry = apply(acc, __shfl_sync(0xffffffffu, xval, first));
+        break;
       }
+      base += BACKWARD ? 32 : -32;
     }
-    if (!resolved) carry = acc.b;  // ran past the array end: nothing enters
   }
-  if (!silent && !self_cut) {
-    st_relaxed_u32(&mine->x, to_bits(apply(agg, carry)));
-    st_release_u32(&mine->flag, tag | kDescInclusive);
-  }
+  if (lane == 0 && !silent && !self_cut) st_relaxed_u64(&mine->w[0], desc_word(tag | kDescInclusive, to_bits(apply(agg, carry))));
   return carry;
 }
 

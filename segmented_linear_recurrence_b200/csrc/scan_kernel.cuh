@@ -6,27 +6,34 @@
 // on chip, runs the associative scan on chip and writes each output once, so
 // a call moves each element through HBM exactly once.
 //
-// Work decomposition (ours, B200-first).  A launch sees its [rows, T] slice as
-// one flat sequence of `total` steps cut into chunks of L = 8 * BLOCK steps,
-// one chunk per thread block; thread j of a block owns the 8 consecutive steps
-// starting at chunk * L + 8j (one 256-bit load per fp32 array).  Because the
-// coefficient builders put a = 0 on each row's dependency edge, chunks may
-// straddle rows freely: the flat scan never leaks a value across a row.
+// Work decomposition (ours, B200-first).  Thread j of a block owns the 8
+// consecutive steps starting at base + 8j, base a multiple of 8 (one 256-bit
+// load per fp32 array).  Two plans:
+//   LB == false (rows fit a block): block b owns rows [b k, (b + 1) k), i.e.
+//     the steps [b span, (b + 1) span) with span = k T.  Its tiles start at
+//     that range's first step rounded down to a multiple of 8, so the first
+//     and last tile may hold steps of the neighbouring blocks: those are
+//     loaded (in bounds, harmless) but neither scanned nor stored.  Every
+//     block's range starts and ends on row edges, so no block needs a carry
+//     from another.  The host picks k (and the block size) to fill the
+//     block's threads.
+//   LB == true (rows longer than a block): the launch's steps are one flat
+//     sequence cut into chunks of L = 8 * BLOCK steps; chunks take tickets
+//     in dependency order and hand carries over with a decoupled look-back
+//     (scan_core.cuh).  Because the coefficient builders put a = 0 on each
+//     row's dependency edge, chunks may straddle rows freely: the flat scan
+//     never leaks a value across a row.
 //
 // Memory-level parallelism comes from occupancy: blocks are small in
 // registers, so several per SM have their loads in flight while others scan,
 // and the hardware block scheduler keeps refilling SMs.  Every load whose
-// address follows from the chunk's position (per-step arrays, the halo step,
+// address follows from the tile's position (per-step arrays, the halo step,
 // the bootstrap of a row end) is issued up front; only trunc_value at
 // truncated steps depends on loaded data.
-//   LB == false : the host only picks this when L is a multiple of T, so every
-//                 chunk ends (backward) / starts (forward) on a row edge and
-//                 needs no carry from another chunk.
-//   LB == true  : chunks take tickets in dependency order and hand carries
-//                 over with a decoupled look-back (scan_core.cuh).
 #pragma once
 
 #include <cstdint>
+#include <cstring>
 #include <cuda_runtime.h>
 
 #include "estimators.cuh"
@@ -38,26 +45,30 @@ struct ScanGeom {
   uint32_t total;         // steps in this launch (rows * T)
   uint32_t T;             // steps per row
   uint32_t nchunks;       // chunks (blocks) in this launch
+  uint32_t span;          // rows plan: steps per block (k T)
   uint32_t vec;           // 1: arrays aligned for 256-bit (flags: 64-bit) accesses
   uint32_t div_m, div_l;  // FastDiv by T
-  uint32_t fetch_wrap;    // the ticket counter wraps to 0 after this value
   LookbackCtl lb;         // ticket / done / epoch counters and descriptors (look-back only)
 };
 
-// Steps, row position and row edges of one thread's tile.
+// Steps, row position and row edges of the tile at step i0 (a multiple of 8)
+// of a block that owns the steps [lo, hi), i0 + 8 > lo.
 template <bool BWD>
-__device__ __forceinline__ Tile make_tile(const ScanGeom &g, const FastDiv &fd, uint32_t chunk, uint32_t L,
-                                          int tid) {
+__device__ __forceinline__ Tile make_tile(const ScanGeom &g, const FastDiv &fd, uint32_t i0, uint32_t lo,
+                                          uint32_t hi) {
   Tile t;
-  t.i0 = chunk * L + uint32_t(kTile) * uint32_t(tid);
-  t.nvalid = t.i0 < g.total ? int(min(uint32_t(kTile), g.total - t.i0)) : 0;
-  t.valid = (1u << t.nvalid) - 1u;
+  t.i0 = i0;
+  t.nvalid = i0 < g.total ? int(min(uint32_t(kTile), g.total - i0)) : 0;
+  uint32_t v = i0 < hi ? (1u << min(uint32_t(kTile), hi - i0)) - 1u : 0u;
+  if (i0 < lo) v &= ~((1u << (lo - i0)) - 1u);
+  t.valid = v;
   t.fast = g.vec != 0u && t.nvalid == kTile;
+  t.full = t.fast && v == 0xffu;
   t.few_rows = g.T >= uint32_t(kTile);
   t.n0 = 0;
   t.t0 = 0;
   t.edge = 0;
-  if (t.nvalid == 0) return t;
+  if (v == 0u) return t;
   t.n0 = fd.div(t.i0);
   t.t0 = t.i0 - t.n0 * g.T;
   uint32_t e = 0;
@@ -81,8 +92,48 @@ __device__ __forceinline__ Tile make_tile(const ScanGeom &g, const FastDiv &fd, 
   return t;
 }
 
+// Word-wise copy of a register-resident value to / from column `lane` of a
+// [words][32] shared array (conflict-free).  Warp 0 parks its tile state
+// there while it runs the look-back, so the look-back's registers do not add
+// to the tile's.
+template <class T>
+__device__ __forceinline__ void park(uint32_t (*s)[32], int lane, const T &v) {
+  static_assert(sizeof(T) % 4 == 0, "parked values are whole words");
+#pragma unroll
+  for (int i = 0; i < int(sizeof(T) / 4); ++i) {
+    uint32_t u;
+    memcpy(&u, reinterpret_cast<const char *>(&v) + 4 * i, 4);
+    s[i][lane] = u;
+  }
+}
+template <class T>
+__device__ __forceinline__ void unpark(const uint32_t (*s)[32], int lane, T &v) {
+#pragma unroll
+  for (int i = 0; i < int(sizeof(T) / 4); ++i) {
+    const uint32_t u = s[i][lane];
+    memcpy(reinterpret_cast<char *>(&v) + 4 * i, &u, 4);
+  }
+}
+
+// Blocks per SM the register budget must allow: each estimator states the
+// registers per thread its tile needs (Op::kRegs, and Op::kRegsLookback for
+// the look-back kernel, whose walk runs in warp 0 only and may spill there).
+// More resident blocks keep more loads in flight.  The register file is four
+// 16K-register partitions, one per warp scheduler, so the count is the most
+// blocks whose warps, spread over the four, each get `regs` (rounded up to
+// the allocation unit of 8).
 template <class Op, int BLOCK, bool LB>
-__global__ void __launch_bounds__(BLOCK, 1024 / BLOCK) scan_kernel(const typename Op::Args p, const ScanGeom g) {
+constexpr int min_blocks_per_sm() {
+  constexpr int regs = ((LB ? Op::kRegsLookback : Op::kRegs) + 7) / 8 * 8;
+  constexpr int warps = BLOCK / 32;
+  int b = 2048 / BLOCK;
+  while (b > 1 && ((b * warps + 3) / 4) * 32 * regs > 16384) --b;
+  return b;
+}
+
+template <class Op, int BLOCK, bool LB>
+__global__ void __launch_bounds__(BLOCK, (min_blocks_per_sm<Op, BLOCK, LB>()))
+    scan_kernel(const typename Op::Args p, const ScanGeom g) {
   using V = typename Op::V;
   using Raw = typename Op::Raw;
   constexpr bool BWD = Op::kBackward;
@@ -93,34 +144,46 @@ __global__ void __launch_bounds__(BLOCK, 1024 / BLOCK) scan_kernel(const typenam
   __shared__ Aff<V> s_wagg[W];
   __shared__ V s_wcarry[W];
   __shared__ uint32_t s_ticket, s_epoch;
+  constexpr int kParked = LB ? int((sizeof(Raw) + sizeof(Aff<V>) * kTile) / 4) : 1;
+  __shared__ uint32_t s_park[kParked][32];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const FastDiv fd{g.div_m, g.div_l};
+  // With programmatic dependent launch this grid may start while the previous
+  // kernel on the stream finishes; wait for it before touching memory.
+  grid_dependency_wait();
 
   // Chunk selection.  With look-back, tickets go out in dependency order
   // (backward: the highest chunk first), so whatever a block waits for is
-  // owned by a block that has already started.  atomicInc wraps the counter
-  // back to 0 after the launch's last ticket.
+  // owned by a block that has already started.
   uint32_t chunk = blockIdx.x, ticket = 0, epoch = 0;
   if constexpr (LB) {
-    if (tid == 0) {
-      s_ticket = atomicInc(&g.lb.hdr->ticket, g.fetch_wrap);
-      s_epoch = *reinterpret_cast<volatile uint32_t *>(&g.lb.hdr->epoch);
-    }
+    if (tid == 0 && !draw_ticket(g.lb.hdr, g.nchunks, s_ticket, s_epoch)) record_status(kDevStatusTimeout);
     __syncthreads();
     ticket = s_ticket;
     epoch = s_epoch;
-    if (ticket >= g.nchunks) {  // counter left inconsistent by an aborted launch
-      if (tid == 0) record_status(kDevStatusTimeout);
-      return;
-    }
+    if (ticket >= g.nchunks) return;  // counter left inconsistent by an aborted launch
     chunk = BWD ? g.nchunks - 1u - ticket : ticket;
   }
 
+  // The block's steps [lo, hi) and its tiles' base.
+  uint32_t lo, hi, base;
+  if constexpr (LB) {
+    lo = chunk * L;
+    hi = min(lo + L, g.total);
+    base = lo;
+  } else {
+    lo = chunk * g.span;
+    hi = min(lo + g.span, g.total);
+    base = lo & ~uint32_t(kTile - 1);
+  }
+
   // a1: every position-determined load of the tile goes out together.
-  const Tile tl = make_tile<BWD>(g, fd, chunk, L, tid);
+  const Tile tl = make_tile<BWD>(g, fd, base + uint32_t(kTile) * uint32_t(tid), lo, hi);
   Raw w;
   Op::load(p, tl, fd, lane, g.total, w);
+  // Every block has issued its loads: the next kernel may start launching.
+  grid_dependents_launch();
 
   // Neighbouring step across the lane edge (t+1 backward, t-1 forward).
   auto mine = Op::nbr_of(w);
@@ -130,9 +193,11 @@ __global__ void __launch_bounds__(BLOCK, 1024 / BLOCK) scan_kernel(const typenam
   // a2: coefficients in registers.
   Aff<V> c[kTile];
   Op::coef(p, tl, fd, w, from, c);
+  if (tl.valid != 0xffu) {
 #pragma unroll
-  for (int k = 0; k < kTile; ++k)
-    if (!((tl.valid >> k) & 1u)) c[k] = aff_identity<V>();
+    for (int k = 0; k < kTile; ++k)
+      if (!((tl.valid >> k) & 1u)) c[k] = aff_identity<V>();
+  }
 
   // a4: sequential composite of the thread's 8 steps, in dependency order.
   Aff<V> agg;
@@ -162,12 +227,16 @@ __global__ void __launch_bounds__(BLOCK, 1024 / BLOCK) scan_kernel(const typenam
     if constexpr (LB) {
       const V ca = __shfl_sync(0xffffffffu, winc.a, BWD ? 0 : W - 1);
       const V cb = __shfl_sync(0xffffffffu, winc.b, BWD ? 0 : W - 1);
-      if (lane == 0) {
-        const uint32_t cbase = chunk * L;
-        const bool edge_closed = BWD ? (min(cbase + L, g.total) % g.T) == 0u : (cbase % g.T) == 0u;
-        carry = decoupled_lookback<BWD, V>(g.lb, chunk, g.nchunks, epoch, ticket, Aff<V>{ca, cb}, edge_closed);
-      }
-      carry = __shfl_sync(0xffffffffu, carry, 0);
+      park(s_park, lane, w);
+      park(s_park + sizeof(Raw) / 4, lane, c);
+      // Re-read from shared memory rather than kept live through the loads.
+      const uint32_t tk = *reinterpret_cast<volatile uint32_t *>(&s_ticket);
+      const uint32_t ep = *reinterpret_cast<volatile uint32_t *>(&s_epoch);
+      const uint32_t ch = BWD ? g.nchunks - 1u - tk : tk;
+      const bool edge_closed = BWD ? (min((ch + 1u) * L, g.total) % g.T) == 0u : ((ch * L) % g.T) == 0u;
+      carry = decoupled_lookback<BWD, V>(g.lb, ch, g.nchunks, ep, tk, Aff<V>{ca, cb}, edge_closed, lane);
+      unpark(s_park, lane, w);
+      unpark(s_park + sizeof(Raw) / 4, lane, c);
     }
     if (lane < W) s_wcarry[lane] = apply(wexc, carry);
   }
@@ -192,16 +261,6 @@ __global__ void __launch_bounds__(BLOCK, 1024 / BLOCK) scan_kernel(const typenam
     }
   }
   Op::emit(p, tl, w, c, xs, xd);
-
-  if constexpr (LB) {
-    // The last block of the launch advances the epoch (its done counter wraps
-    // to 0 by itself); every block has read the epoch and finished its
-    // look-back before it counts itself done.
-    if (tid == 0) {
-      __threadfence();
-      if (atomicInc(&g.lb.hdr->done, g.nchunks - 1u) == g.nchunks - 1u) atomicAdd(&g.lb.hdr->epoch, 1u);
-    }
-  }
 }
 
 }  // namespace rlscan

@@ -137,8 +137,18 @@ def test_query_plan(L):
     assert p["lookback"] == 1 and p["workspace_bytes"] >= 16 * p["chunks"]
     p = slr.rlscan_query_plan("retrace", 2048, 512, 18)
     assert p["lookback"] == 0 and p["block_threads"] in (128, 256)
+    # rows that do not divide a block still get whole-row blocks
     p = slr.rlscan_query_plan("episodic_prefix_sum", 3, 33)
-    assert p["lookback"] == 1
+    assert p["lookback"] == 0 and p["chunk_steps"] % 33 == 0 and p["chunks"] == 1
+    p = slr.rlscan_query_plan("gae", 4096, 2000)
+    assert p["lookback"] == 0 and p["chunk_steps"] % 2000 == 0
+    assert p["chunks"] == -(-4096 // (p["chunk_steps"] // 2000))
+    # the block size whose threads whole rows fill best
+    assert slr.rlscan_query_plan("gae", 64, 3000)["block_threads"] == 384
+    assert slr.rlscan_query_plan("gae", 64, 1500)["block_threads"] == 192
+    # a row longer than the largest block needs the look-back
+    assert slr.rlscan_query_plan("gae", 8, 4097)["lookback"] == 1
+    assert slr.rlscan_query_plan("gae", 8, 4096)["lookback"] == 0
     # more steps than one launch takes are split by rows
     p = slr.rlscan_query_plan("discounted_return", 1 << 12, 1 << 19)
     assert p["launches"] == 2
@@ -148,12 +158,15 @@ def test_query_plan(L):
 def test_options_roundtrip(L):
     for name, default in (("lookback_timeout_ns", 10 ** 9), ("force_lookback", 0),
                           ("force_block", 0), ("force_scalar", 0), ("check_pointers", 1),
-                          ("test_starve_lookback", 0)):
+                          ("test_starve_lookback", 0), ("pdl", 1)):
         assert slr.rlscan_get_option(name) == default
     slr.rlscan_set_option("force_block", 512)
     assert slr.rlscan_query_plan("gae", 64, 32)["block_threads"] == 512
     slr.rlscan_set_option("force_block", 0)
-    for bad in (100, 1024):
+    slr.rlscan_set_option("force_block", 192)
+    assert slr.rlscan_query_plan("gae", 64, 32)["block_threads"] == 192
+    slr.rlscan_set_option("force_block", 0)
+    for bad in (100, 200, 576, 1024):
         with pytest.raises(slr.RlscanError):
             slr.rlscan_set_option("force_block", bad)
     with pytest.raises(slr.RlscanError):

@@ -31,18 +31,19 @@ def _built():
 def options():
     yield slr.rlscan_set_option
     for name, default in (("force_lookback", 0), ("force_block", 0), ("force_scalar", 0),
-                          ("test_starve_lookback", 0), ("lookback_timeout_ns", 10 ** 9)):
+                          ("test_starve_lookback", 0), ("lookback_timeout_ns", 10 ** 9),
+                          ("pdl", 1)):
         slr.rlscan_set_option(name, default)
 
 
-PLAN_CASES = [(4096 // 8, 128), (64, 2048), (5, 5000), (40, 96)]
+PLAN_CASES = [(4096 // 8, 128), (64, 2048), (5, 5000), (40, 96), (33, 1001), (7, 3)]
 
 
 @pytest.mark.parametrize("est", synthetic.ESTIMATORS)
-@pytest.mark.parametrize("block", [128, 256, 512])
+@pytest.mark.parametrize("block", [128, 192, 256, 320, 384, 448, 512])
 @pytest.mark.parametrize("lookback", [0, 1])
 def test_every_plan_matches_oracle(est, block, lookback, options):
-    if est == "retrace" and block > 256:
+    if est == "retrace" and block not in (128, 256):
         pytest.skip("Retrace stages its action rows with 128- or 256-thread blocks")
     options("force_block", block)
     options("force_lookback", lookback)
@@ -50,7 +51,7 @@ def test_every_plan_matches_oracle(est, block, lookback, options):
         d = synthetic.make_inputs(est, N, T, seed=900 + N + T, p_term=0.01, p_trunc=0.01, A=6,
                                   with_init=True)
         plan = slr.rlscan_query_plan(est, N, T, 6)
-        assert plan["block_threads"] == (block if est != "retrace" or block <= 256 else 128)
+        assert plan["block_threads"] == block
         if lookback:
             assert plan["lookback"] == 1
         check(est, d, synthetic.SCALARS[est], what=f"block={block} lookback={lookback} N={N} T={T}")
@@ -67,6 +68,21 @@ def test_scalar_path_matches_vector_path(est, options):
     for a, b in zip(vec, sca):
         if a is not None:
             np.testing.assert_array_equal(a, b)
+
+
+@pytest.mark.parametrize("est", synthetic.ESTIMATORS)
+def test_plain_launch_matches_programmatic_launch(est, options):
+    # back-to-back calls with and without programmatic dependent launch
+    d = synthetic.make_inputs(est, 96, 700, seed=70, p_term=0.01, p_trunc=0.01, A=6,
+                              with_init=True)
+    s = f32_scalars(est, synthetic.SCALARS[est])
+    pdl = [gpu_run(est, d, **s) for _ in range(3)]
+    options("pdl", 0)
+    plain = gpu_run(est, d, **s)
+    for run in pdl:
+        for a, b in zip(run, plain):
+            if a is not None:
+                np.testing.assert_array_equal(a, b)
 
 
 def test_lookback_survives_many_calls_on_one_stream(options):

@@ -15,14 +15,16 @@
 // array, one 64-bit load per flag array.  Interface used by scan_kernel.cuh
 // (all members static __device__):
 //   V, kBackward, Args, Raw
-//   load(args, tile, lane, total, raw)   issues every load whose address is
-//        known from the tile's position alone: the per-step arrays, the halo
-//        step across the lane edge (lane 31 backward / lane 0 forward) and the
+//   load(args, tile, fd, lane, total, flags, raw)   given the tile's
+//        terminated / truncated masks, issues every load whose address
+//        follows from the tile's position: the per-step arrays, the halo step
+//        across the lane edge (lane 31 backward / lane 0 forward) and the
 //        per-row value (bootstrap / initial trace) of the tile's row edge
+//   fetch_boundary(args, tile, raw)      issues the loads that depend on the
+//        flags (trunc_value at truncated steps, backward estimators)
 //   nbr_of(raw) / halo_of(raw)           the step a neighbouring lane needs
-//   coef(args, tile, fd, raw, nbr, c)    fills the 8 coefficients; the only
-//        data-dependent loads (trunc_value where truncated) are issued here;
-//        may keep per-step state in `raw` for emit()
+//   coef(args, tile, fd, raw, nbr, c)    fills the 8 coefficients; may keep
+//        per-step state in `raw` for emit()
 //   emit(args, tile, raw, c, x, xdep)    writes the outputs
 // x[k] is the solved value at step k, xdep[k] the one it was derived from
 // (x_{t+1} backward, x_{t-1} forward).
@@ -129,25 +131,31 @@ __device__ __forceinline__ float edge_value(const float *src, const Tile &tl, co
   return __ldg(src + tl.n0 + fd.div(tl.t0 + k));
 }
 
-// Successor values of the tile's boundary steps (backward estimators): 0 after
-// termination, trunc_value after truncation (the only loads that depend on the
-// data), the row's bootstrap at a row end.
-__device__ __forceinline__ void boundary_values(const float *tv, const float *boot, float edge_val, const Tile &tl,
-                                                uint32_t term, uint32_t trunc, const FastDiv &fd, float (&sv)[8]) {
-  const uint32_t tr = trunc & ~term & tl.valid;
-  const uint32_t ed = tl.edge & ~term & ~trunc;
+// Terminated / truncated masks of a tile (bit k: step k).
+struct Flags {
+  uint32_t term, trunc;
+};
+
+// trunc_value at the tile's truncated (not terminated) steps: the only loads
+// whose addresses depend on loaded data.  Warps without such a step skip them.
+__device__ __forceinline__ void trunc_values(const float *tv, const Tile &tl, Flags f, float (&sv)[8]) {
+  const uint32_t tr = f.trunc & ~f.term & tl.valid;
 #pragma unroll
   for (int k = 0; k < 8; ++k) sv[k] = 0.0f;
-  if (!__any_sync(0xffffffffu, (tr | ed) != 0u)) return;  // most warps: nothing to fetch
+  if (!__any_sync(0xffffffffu, tr != 0u)) return;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    float s = 0.0f;
-    if ((tr >> k) & 1u)
-      s = __ldg(tv + tl.i0 + k);
-    else if ((ed >> k) & 1u)
-      s = tl.few_rows ? edge_val : (boot ? __ldg(boot + tl.n0 + fd.div(tl.t0 + k)) : 0.0f);
-    sv[k] = s;
-  }
+  for (int k = 0; k < 8; ++k)
+    if ((tr >> k) & 1u) sv[k] = __ldg(tv + tl.i0 + k);
+}
+
+// Successor value of boundary step k (backward estimators): 0 after
+// termination, trunc_value after truncation, the row's bootstrap at a row end
+// (`boot` may be NULL: 0).
+__device__ __forceinline__ float boundary_value(int k, Flags f, const float (&sv)[8], float ev, const float *boot,
+                                                const Tile &tl, const FastDiv &fd) {
+  if ((f.term >> k) & 1u) return 0.0f;
+  if ((f.trunc >> k) & 1u) return sv[k];
+  return tl.few_rows ? ev : (boot ? __ldg(boot + tl.n0 + fd.div(tl.t0 + k)) : 0.0f);
 }
 
 // ---------------------------------------------------------------------------
@@ -155,7 +163,7 @@ __device__ __forceinline__ void boundary_values(const float *tv, const float *bo
 // b = r + gamma nv - v.  Outputs advantages = x, returns = x + v.
 // ---------------------------------------------------------------------------
 struct GaeOp {
-  static constexpr int kRegs = 40, kRegsLookback = 48;  // registers per thread (see scan_kernel.cuh)
+  static constexpr int kRegs = 48, kRegsLookback = 48;  // registers per thread, chosen by measurement
   using V = float;
   static constexpr bool kBackward = true;
   struct Args {
@@ -165,32 +173,32 @@ struct GaeOp {
     float gamma, gl;
   };
   struct Raw {
-    float r[8], v[8];
-    uint32_t term, trunc;
+    float r[8], v[8], sv[8];  // sv: trunc_value at truncated steps
+    Flags f;
     float halo;  // v of the step after the tile (lane 31 only)
     float ev;    // bootstrap of the tile's row end
   };
   static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int lane,
-                                              uint32_t total, Raw &w) {
+                                              uint32_t total, Flags f, Raw &w) {
     ld8(p.r, tl, w.r);
     ld8(p.v, tl, w.v);
-    w.term = ld8_flags(p.term, tl);
-    w.trunc = ld8_flags(p.trunc, tl);
+    w.f = f;
     w.halo = (lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total) ? __ldg(p.v + tl.i0 + 8u) : 0.0f;
     w.ev = edge_value(p.boot, tl, fd);
+  }
+  static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, Raw &w) {
+    trunc_values(p.tv, tl, w.f, w.sv);
   }
   static __device__ __forceinline__ float nbr_of(const Raw &w) { return w.v[0]; }
   static __device__ __forceinline__ float halo_of(const Raw &w) { return w.halo; }
   static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w,
                                               float next7, Aff<float> (&c)[8]) {
-    float sv[8];
-    boundary_values(p.tv, p.boot, w.ev, tl, w.term, w.trunc, fd, sv);
-    const uint32_t special = w.term | w.trunc | tl.edge;
+    const uint32_t special = w.f.term | w.f.trunc | tl.edge;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const bool sp = (special >> k) & 1u;
       const float next = k < 7 ? w.v[k < 7 ? k + 1 : 7] : next7;
-      const float nv = sp ? sv[k] : next;
+      const float nv = sp ? boundary_value(k, w.f, w.sv, w.ev, p.boot, tl, fd) : next;
       c[k] = Aff<float>{sp ? 0.0f : p.gl, fmaf(p.gamma, nv, w.r[k]) - w.v[k]};
     }
   }
@@ -211,7 +219,7 @@ struct GaeOp {
 // inside an episode, b = r + gamma nv at a boundary.  Output x.
 // ---------------------------------------------------------------------------
 struct TdLambdaOp {
-  static constexpr int kRegs = 40, kRegsLookback = 48;  // registers per thread (see scan_kernel.cuh)
+  static constexpr int kRegs = 48, kRegsLookback = 48;  // registers per thread, chosen by measurement
   using V = float;
   static constexpr bool kBackward = true;
   struct Args {
@@ -221,31 +229,32 @@ struct TdLambdaOp {
     float gamma, gl, g1l;  // gamma, gamma*lambda, gamma*(1-lambda)
   };
   struct Raw {
-    float r[8], v[8];
-    uint32_t term, trunc;
+    float r[8], v[8], sv[8];
+    Flags f;
     float halo, ev;
   };
   static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int lane,
-                                              uint32_t total, Raw &w) {
+                                              uint32_t total, Flags f, Raw &w) {
     ld8(p.r, tl, w.r);
     ld8(p.v, tl, w.v);
-    w.term = ld8_flags(p.term, tl);
-    w.trunc = ld8_flags(p.trunc, tl);
+    w.f = f;
     w.halo = (lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total) ? __ldg(p.v + tl.i0 + 8u) : 0.0f;
     w.ev = edge_value(p.boot, tl, fd);
+  }
+  static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, Raw &w) {
+    trunc_values(p.tv, tl, w.f, w.sv);
   }
   static __device__ __forceinline__ float nbr_of(const Raw &w) { return w.v[0]; }
   static __device__ __forceinline__ float halo_of(const Raw &w) { return w.halo; }
   static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w,
                                               float next7, Aff<float> (&c)[8]) {
-    float sv[8];
-    boundary_values(p.tv, p.boot, w.ev, tl, w.term, w.trunc, fd, sv);
-    const uint32_t special = w.term | w.trunc | tl.edge;
+    const uint32_t special = w.f.term | w.f.trunc | tl.edge;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const bool sp = (special >> k) & 1u;
       const float next = k < 7 ? w.v[k < 7 ? k + 1 : 7] : next7;
-      c[k] = sp ? Aff<float>{0.0f, fmaf(p.gamma, sv[k], w.r[k])} : Aff<float>{p.gl, fmaf(p.g1l, next, w.r[k])};
+      c[k] = sp ? Aff<float>{0.0f, fmaf(p.gamma, boundary_value(k, w.f, w.sv, w.ev, p.boot, tl, fd), w.r[k])}
+                : Aff<float>{p.gl, fmaf(p.g1l, next, w.r[k])};
     }
   }
   static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[8],
@@ -259,7 +268,7 @@ struct TdLambdaOp {
 // bootstrap may be NULL (zero at the window end).  Output x.
 // ---------------------------------------------------------------------------
 struct DiscountedOp {
-  static constexpr int kRegs = 32, kRegsLookback = 48;  // registers per thread (see scan_kernel.cuh)
+  static constexpr int kRegs = 32, kRegsLookback = 40;  // registers per thread, chosen by measurement
   using V = float;
   static constexpr bool kBackward = true;
   struct Args {
@@ -269,28 +278,29 @@ struct DiscountedOp {
     float gamma;
   };
   struct Raw {
-    float r[8];
-    uint32_t term, trunc;
+    float r[8], sv[8];
+    Flags f;
     float ev;
   };
   static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int, uint32_t,
-                                              Raw &w) {
+                                              Flags f, Raw &w) {
     ld8(p.r, tl, w.r);
-    w.term = ld8_flags(p.term, tl);
-    w.trunc = ld8_flags(p.trunc, tl);
+    w.f = f;
     w.ev = edge_value(p.boot, tl, fd);
+  }
+  static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, Raw &w) {
+    trunc_values(p.tv, tl, w.f, w.sv);
   }
   static __device__ __forceinline__ float nbr_of(const Raw &) { return 0.0f; }
   static __device__ __forceinline__ float halo_of(const Raw &) { return 0.0f; }
   static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w, float,
                                               Aff<float> (&c)[8]) {
-    float sv[8];
-    boundary_values(p.tv, p.boot, w.ev, tl, w.term, w.trunc, fd, sv);
-    const uint32_t special = w.term | w.trunc | tl.edge;
+    const uint32_t special = w.f.term | w.f.trunc | tl.edge;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const bool sp = (special >> k) & 1u;
-      c[k] = sp ? Aff<float>{0.0f, fmaf(p.gamma, sv[k], w.r[k])} : Aff<float>{p.gamma, w.r[k]};
+      c[k] = sp ? Aff<float>{0.0f, fmaf(p.gamma, boundary_value(k, w.f, w.sv, w.ev, p.boot, tl, fd), w.r[k])}
+                : Aff<float>{p.gamma, w.r[k]};
     }
   }
   static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[8],
@@ -307,7 +317,7 @@ struct DiscountedOp {
 // episode (vs_{t+1} = v_{t+1} + x_{t+1}), rho (r + gamma nv - v) at a boundary.
 // ---------------------------------------------------------------------------
 struct VtraceOp {
-  static constexpr int kRegs = 48, kRegsLookback = 56;  // registers per thread (see scan_kernel.cuh)
+  static constexpr int kRegs = 56, kRegsLookback = 48;  // registers per thread, chosen by measurement
   using V = float;
   static constexpr bool kBackward = true;
   struct Args {
@@ -317,32 +327,32 @@ struct VtraceOp {
     float gamma, lambda, rho_bar, c_bar;
   };
   struct Raw {
-    float lr[8], r[8], v[8];  // coef() keeps gamma * rho * cont in lr for emit()
-    uint32_t term, trunc;
+    float lr[8], r[8], v[8], sv[8];  // coef() keeps gamma * rho * cont in lr for emit()
+    Flags f;
     float halo, ev;
   };
   static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int lane,
-                                              uint32_t total, Raw &w) {
+                                              uint32_t total, Flags f, Raw &w) {
     ld8(p.lr, tl, w.lr);
     ld8(p.r, tl, w.r);
     ld8(p.v, tl, w.v);
-    w.term = ld8_flags(p.term, tl);
-    w.trunc = ld8_flags(p.trunc, tl);
+    w.f = f;
     w.halo = (lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total) ? __ldg(p.v + tl.i0 + 8u) : 0.0f;
     w.ev = edge_value(p.boot, tl, fd);
+  }
+  static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, Raw &w) {
+    trunc_values(p.tv, tl, w.f, w.sv);
   }
   static __device__ __forceinline__ float nbr_of(const Raw &w) { return w.v[0]; }
   static __device__ __forceinline__ float halo_of(const Raw &w) { return w.halo; }
   static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w,
                                               float next7, Aff<float> (&c)[8]) {
-    float sv[8];
-    boundary_values(p.tv, p.boot, w.ev, tl, w.term, w.trunc, fd, sv);
-    const uint32_t special = w.term | w.trunc | tl.edge;
+    const uint32_t special = w.f.term | w.f.trunc | tl.edge;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const bool sp = (special >> k) & 1u;
       const float next = k < 7 ? w.v[k < 7 ? k + 1 : 7] : next7;
-      const float nv = sp ? sv[k] : next;
+      const float nv = sp ? boundary_value(k, w.f, w.sv, w.ev, p.boot, tl, fd) : next;
       const float ratio = __expf(w.lr[k]);
       const float rho = fminf(p.rho_bar, ratio);
       const float cc = p.lambda * fminf(p.c_bar, ratio);
@@ -370,7 +380,7 @@ struct VtraceOp {
 // b = g + gamma lambda init[n], a = 0.  Output x.
 // ---------------------------------------------------------------------------
 struct EligOp {
-  static constexpr int kRegs = 32, kRegsLookback = 48;  // registers per thread (see scan_kernel.cuh)
+  static constexpr int kRegs = 40, kRegsLookback = 32;  // registers per thread, chosen by measurement
   using V = float;
   static constexpr bool kBackward = false;
   struct Args {
@@ -386,14 +396,15 @@ struct EligOp {
     float ev;       // initial trace of the tile's row start
   };
   static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int lane, uint32_t,
-                                              Raw &w) {
+                                              Flags f, Raw &w) {
     ld8(p.g, tl, w.g);
-    w.done = ld8_flags(p.term, tl) | ld8_flags(p.trunc, tl);
+    w.done = f.term | f.trunc;
     w.halo = 0u;
     if (lane == 0 && tl.i0 > 0u && tl.nvalid > 0)
       w.halo = ((p.term && __ldg(p.term + tl.i0 - 1u)) || (p.trunc && __ldg(p.trunc + tl.i0 - 1u))) ? 1u : 0u;
     w.ev = edge_value(p.init, tl, fd);
   }
+  static __device__ __forceinline__ void fetch_boundary(const Args &, const Tile &, Raw &) {}
   static __device__ __forceinline__ uint32_t nbr_of(const Raw &w) { return (w.done >> 7) & 1u; }
   static __device__ __forceinline__ uint32_t halo_of(const Raw &w) { return w.halo; }
   static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w,
@@ -418,7 +429,7 @@ struct EligOp {
 // a = 0 at a row start or after a done step, else 1; b = x.
 // ---------------------------------------------------------------------------
 struct PrefixSumOp {
-  static constexpr int kRegs = 32, kRegsLookback = 48;  // registers per thread (see scan_kernel.cuh)
+  static constexpr int kRegs = 40, kRegsLookback = 32;  // registers per thread, chosen by measurement
   using V = uint32_t;
   static constexpr bool kBackward = false;
   struct Args {
@@ -432,13 +443,14 @@ struct PrefixSumOp {
     uint32_t halo;
   };
   static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &, int lane, uint32_t,
-                                              Raw &w) {
+                                              Flags f, Raw &w) {
     ld8(p.x, tl, w.x);
-    w.done = ld8_flags(p.term, tl) | ld8_flags(p.trunc, tl);
+    w.done = f.term | f.trunc;
     w.halo = 0u;
     if (lane == 0 && tl.i0 > 0u && tl.nvalid > 0)
       w.halo = ((p.term && __ldg(p.term + tl.i0 - 1u)) || (p.trunc && __ldg(p.trunc + tl.i0 - 1u))) ? 1u : 0u;
   }
+  static __device__ __forceinline__ void fetch_boundary(const Args &, const Tile &, Raw &) {}
   static __device__ __forceinline__ uint32_t nbr_of(const Raw &w) { return (w.done >> 7) & 1u; }
   static __device__ __forceinline__ uint32_t halo_of(const Raw &w) { return w.halo; }
   static __device__ __forceinline__ void coef(const Args &, const Tile &tl, const FastDiv &, Raw &w, uint32_t prev7,

@@ -306,9 +306,36 @@ void fast_div_params(uint32_t d, uint32_t &m, uint32_t &l) {
   m = uint32_t(((uint64_t(1) << (31 + l)) + d - 1) / d);
 }
 
+// Blocks of `kern` that fit on the current device at once (occupancy x SMs),
+// cached per (device, kernel).
+int resident_blocks(const void *kern, int block) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  static std::mutex mu;
+  static std::map<std::pair<int, const void *>, int> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(dev, kern);
+  const auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int per_sm = 0, sms = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, block, 0) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 1;
+  }
+  const int n = std::max(1, per_sm * sms);
+  cache[key] = n;
+  return n;
+}
+
+// Look-back plan: one block per chunk.  Rows plan: persistent blocks, as
+// many as fit at once, each taking every gridDim-th chunk.
 template <class Op, int BLOCK, bool LB>
 cudaError_t launch_scan(const typename Op::Args &a, ScanGeom g, cudaStream_t s) {
-  const cudaError_t e = launch(scan_kernel<Op, BLOCK, LB>, g.nchunks, BLOCK, 0, s, a, g);
+  auto kern = scan_kernel<Op, BLOCK, LB>;
+  uint32_t grid = g.nchunks;
+  if (!LB) grid = std::min<uint32_t>(grid, uint32_t(resident_blocks(reinterpret_cast<const void *>(kern), BLOCK)));
+  const cudaError_t e = launch(kern, grid, BLOCK, 0, s, a, g);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -93,7 +93,7 @@ __device__ __forceinline__ Tile make_tile(const ScanGeom &g, const FastDiv &fd, 
 }
 
 // Word-wise copy of a register-resident value to / from column `lane` of a
-// [words][32] shared array (conflict-free).  Warp 0 parks its tile state
+// [words][32] shared array (conflict-free).  Warp 0 parks its coefficients
 // there while it runs the look-back, so the look-back's registers do not add
 // to the tile's.
 template <class T>
@@ -131,57 +131,53 @@ constexpr int min_blocks_per_sm() {
   return b;
 }
 
+// Flag bytes of one tile, prefetched into shared memory for the block's next
+// chunk: each thread copies its own tile's 8 terminated and 8 truncated bytes
+// with cp.async and reads them back itself (no barrier needed).
+struct FlagSlot {
+  uint32_t term[2], trunc[2];
+};
+
+__device__ __forceinline__ void cp_async8(void *dst_smem, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst_smem))),
+               "l"(src)
+               : "memory");
+}
+
+// Shared state of one block, reused chunk after chunk.
 template <class Op, int BLOCK, bool LB>
-__global__ void __launch_bounds__(BLOCK, (min_blocks_per_sm<Op, BLOCK, LB>()))
-    scan_kernel(const typename Op::Args p, const ScanGeom g) {
+struct ScanSmem {
+  using V = typename Op::V;
+  static constexpr int W = BLOCK / 32;
+  static constexpr int kParked = LB ? int(sizeof(Aff<V>) * kTile / 4) : 1;
+  Aff<V> wagg[W];
+  V wcarry[W];
+  uint32_t ticket, epoch;
+  uint32_t park[kParked][32];
+};
+
+// One chunk: the block's steps [lo, hi), tiles from `base`.  `f` holds the
+// thread's flag masks.  Look-back plan: `chunk` is the ticketed chunk.
+// Rows plan: the loads that depend on the flags go out right behind the
+// tile's other loads (the flags are normally in hand already, prefetched).
+// Look-back plan: they follow once the tile's own loads have arrived, which
+// keeps their registers out of the load phase.
+template <class Op, int BLOCK, bool LB>
+__device__ __forceinline__ void scan_chunk(const typename Op::Args &p, const ScanGeom &g, const FastDiv &fd,
+                                           ScanSmem<Op, BLOCK, LB> &sm, uint32_t chunk, const Tile &tl, Flags f,
+                                           int tid) {
+  constexpr bool early = !LB;
   using V = typename Op::V;
   using Raw = typename Op::Raw;
   constexpr bool BWD = Op::kBackward;
   constexpr int W = BLOCK / 32;
   constexpr uint32_t L = uint32_t(kTile) * BLOCK;
-  static_assert(BLOCK % 32 == 0 && W <= 32, "block must be whole warps, at most 32");
+  const int lane = tid & 31, warp = tid >> 5;
 
-  __shared__ Aff<V> s_wagg[W];
-  __shared__ V s_wcarry[W];
-  __shared__ uint32_t s_ticket, s_epoch;
-  constexpr int kParked = LB ? int((sizeof(Raw) + sizeof(Aff<V>) * kTile) / 4) : 1;
-  __shared__ uint32_t s_park[kParked][32];
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const FastDiv fd{g.div_m, g.div_l};
-  // With programmatic dependent launch this grid may start while the previous
-  // kernel on the stream finishes; wait for it before touching memory.
-  grid_dependency_wait();
-
-  // Chunk selection.  With look-back, tickets go out in dependency order
-  // (backward: the highest chunk first), so whatever a block waits for is
-  // owned by a block that has already started.
-  uint32_t chunk = blockIdx.x, ticket = 0, epoch = 0;
-  if constexpr (LB) {
-    if (tid == 0 && !draw_ticket(g.lb.hdr, g.nchunks, s_ticket, s_epoch)) record_status(kDevStatusTimeout);
-    __syncthreads();
-    ticket = s_ticket;
-    epoch = s_epoch;
-    if (ticket >= g.nchunks) return;  // counter left inconsistent by an aborted launch
-    chunk = BWD ? g.nchunks - 1u - ticket : ticket;
-  }
-
-  // The block's steps [lo, hi) and its tiles' base.
-  uint32_t lo, hi, base;
-  if constexpr (LB) {
-    lo = chunk * L;
-    hi = min(lo + L, g.total);
-    base = lo;
-  } else {
-    lo = chunk * g.span;
-    hi = min(lo + g.span, g.total);
-    base = lo & ~uint32_t(kTile - 1);
-  }
-
-  // a1: every position-determined load of the tile goes out together.
-  const Tile tl = make_tile<BWD>(g, fd, base + uint32_t(kTile) * uint32_t(tid), lo, hi);
+  // a1: every load of the tile goes out together.
   Raw w;
-  Op::load(p, tl, fd, lane, g.total, w);
+  Op::load(p, tl, fd, lane, g.total, f, w);
+  if constexpr (early) Op::fetch_boundary(p, tl, w);
   // Every block has issued its loads: the next kernel may start launching.
   grid_dependents_launch();
 
@@ -189,6 +185,7 @@ __global__ void __launch_bounds__(BLOCK, (min_blocks_per_sm<Op, BLOCK, LB>()))
   auto mine = Op::nbr_of(w);
   auto from = BWD ? __shfl_down_sync(0xffffffffu, mine, 1) : __shfl_up_sync(0xffffffffu, mine, 1);
   if (BWD ? lane == 31 : lane == 0) from = Op::halo_of(w);
+  if constexpr (!early) Op::fetch_boundary(p, tl, w);
 
   // a2: coefficients in registers.
   Aff<V> c[kTile];
@@ -214,36 +211,33 @@ __global__ void __launch_bounds__(BLOCK, (min_blocks_per_sm<Op, BLOCK, LB>()))
   // a5: warp scan.
   const Aff<V> inc = warp_inclusive_scan<BWD>(agg, lane);
   const Aff<V> exc = warp_exclusive_from_inclusive<BWD>(inc, lane, 31);
-  if (BWD ? lane == 0 : lane == 31) s_wagg[warp] = inc;
+  if (BWD ? lane == 0 : lane == 31) sm.wagg[warp] = inc;
   __syncthreads();
 
-  // a6 (+ a7): warp 0 scans the warp aggregates; with look-back its lane 0
-  // also obtains the carry entering the chunk.
+  // a6 (+ a7): warp 0 scans the warp aggregates; with look-back it also
+  // obtains the carry entering the chunk.
   if (warp == 0) {
-    const Aff<V> wv = lane < W ? s_wagg[lane] : aff_identity<V>();
+    const Aff<V> wv = lane < W ? sm.wagg[lane] : aff_identity<V>();
     const Aff<V> winc = warp_inclusive_scan<BWD>(wv, lane);
     const Aff<V> wexc = warp_exclusive_from_inclusive<BWD>(winc, lane, W - 1);
     V carry = V(0);
     if constexpr (LB) {
       const V ca = __shfl_sync(0xffffffffu, winc.a, BWD ? 0 : W - 1);
       const V cb = __shfl_sync(0xffffffffu, winc.b, BWD ? 0 : W - 1);
-      park(s_park, lane, w);
-      park(s_park + sizeof(Raw) / 4, lane, c);
+      park(sm.park, lane, c);
       // Re-read from shared memory rather than kept live through the loads.
-      const uint32_t tk = *reinterpret_cast<volatile uint32_t *>(&s_ticket);
-      const uint32_t ep = *reinterpret_cast<volatile uint32_t *>(&s_epoch);
-      const uint32_t ch = BWD ? g.nchunks - 1u - tk : tk;
-      const bool edge_closed = BWD ? (min((ch + 1u) * L, g.total) % g.T) == 0u : ((ch * L) % g.T) == 0u;
-      carry = decoupled_lookback<BWD, V>(g.lb, ch, g.nchunks, ep, tk, Aff<V>{ca, cb}, edge_closed, lane);
-      unpark(s_park, lane, w);
-      unpark(s_park + sizeof(Raw) / 4, lane, c);
+      const uint32_t tk = *reinterpret_cast<volatile uint32_t *>(&sm.ticket);
+      const uint32_t ep = *reinterpret_cast<volatile uint32_t *>(&sm.epoch);
+      const bool edge_closed = BWD ? (min((chunk + 1u) * L, g.total) % g.T) == 0u : ((chunk * L) % g.T) == 0u;
+      carry = decoupled_lookback<BWD, V>(g.lb, chunk, g.nchunks, ep, tk, Aff<V>{ca, cb}, edge_closed, lane);
+      unpark(sm.park, lane, c);
     }
-    if (lane < W) s_wcarry[lane] = apply(wexc, carry);
+    if (lane < W) sm.wcarry[lane] = apply(wexc, carry);
   }
   __syncthreads();
 
   // a8: re-sweep the thread's steps from the carry and write the outputs.
-  V x = apply(exc, s_wcarry[warp]);
+  V x = apply(exc, sm.wcarry[warp]);
   V xs[kTile], xd[kTile];
   if (BWD) {
 #pragma unroll
@@ -261,6 +255,76 @@ __global__ void __launch_bounds__(BLOCK, (min_blocks_per_sm<Op, BLOCK, LB>()))
     }
   }
   Op::emit(p, tl, w, c, xs, xd);
+}
+
+template <class Op, int BLOCK, bool LB>
+__global__ void __launch_bounds__(BLOCK, (min_blocks_per_sm<Op, BLOCK, LB>()))
+    scan_kernel(const typename Op::Args p, const ScanGeom g) {
+  constexpr bool BWD = Op::kBackward;
+  constexpr uint32_t L = uint32_t(kTile) * BLOCK;
+  static_assert(BLOCK % 32 == 0 && BLOCK / 32 <= 32, "block must be whole warps, at most 32");
+
+  __shared__ ScanSmem<Op, BLOCK, LB> sm;
+  const int tid = threadIdx.x;
+  const FastDiv fd{g.div_m, g.div_l};
+  // With programmatic dependent launch this grid may start while the previous
+  // kernel on the stream finishes; wait for it before touching memory.
+  grid_dependency_wait();
+
+  if constexpr (LB) {
+    // Chunk selection: tickets go out in dependency order (backward: the
+    // highest chunk first), so whatever a block waits for is owned by a
+    // block that has already started.
+    if (tid == 0 && !draw_ticket(g.lb.hdr, g.nchunks, sm.ticket, sm.epoch)) record_status(kDevStatusTimeout);
+    __syncthreads();
+    const uint32_t ticket = sm.ticket;
+    if (ticket >= g.nchunks) return;  // counter left inconsistent by an aborted launch
+    const uint32_t chunk = BWD ? g.nchunks - 1u - ticket : ticket;
+    const uint32_t lo = chunk * L, hi = min(lo + L, g.total);
+    const Tile tl = make_tile<BWD>(g, fd, lo + uint32_t(kTile) * uint32_t(tid), lo, hi);
+    const Flags f{ld8_flags(p.term, tl), ld8_flags(p.trunc, tl)};
+    scan_chunk<Op, BLOCK, LB>(p, g, fd, sm, chunk, tl, f, tid);
+  } else {
+    // Rows plan, persistent: the block takes chunks blockIdx.x, + gridDim.x,
+    // ...  While it scans one chunk, its threads prefetch the next chunk's
+    // flag bytes, so the trunc_value loads that depend on them go out with
+    // the chunk's other loads instead of a memory round trip later.
+    __shared__ FlagSlot slots[2][BLOCK];
+    auto tile_of = [&](uint32_t chunk) {
+      const uint32_t lo = chunk * g.span, hi = min(lo + g.span, g.total);
+      return make_tile<BWD>(g, fd, (lo & ~uint32_t(kTile - 1)) + uint32_t(kTile) * uint32_t(tid), lo, hi);
+    };
+    // Prefetch needs the 8-byte copies in bounds and aligned: full tiles of
+    // vectorised launches only; any other tile loads its flags directly.
+    // Only the next tile's first step is computed ahead; its full geometry
+    // is built after the current chunk, to keep the loop light in registers.
+    auto prefetch = [&](uint32_t chunk, FlagSlot &slot) {
+      const uint32_t i0 = ((chunk * g.span) & ~uint32_t(kTile - 1)) + uint32_t(kTile) * uint32_t(tid);
+      if (g.vec == 0u || i0 + uint32_t(kTile) > g.total) return false;
+      if (p.term) cp_async8(slot.term, p.term + i0);
+      if (p.trunc) cp_async8(slot.trunc, p.trunc + i0);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      return true;
+    };
+    bool have = false;  // slots[buf][tid] holds this chunk's flags
+    int buf = 0;
+    for (uint32_t chunk = blockIdx.x; chunk < g.nchunks; chunk += gridDim.x) {
+      const Tile tl = tile_of(chunk);
+      Flags f;
+      if (have) {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        const FlagSlot &s = slots[buf][tid];
+        f.term = p.term ? nonzero_bytes4(s.term[0]) | (nonzero_bytes4(s.term[1]) << 4) : 0u;
+        f.trunc = p.trunc ? nonzero_bytes4(s.trunc[0]) | (nonzero_bytes4(s.trunc[1]) << 4) : 0u;
+      } else {
+        f = Flags{ld8_flags(p.term, tl), ld8_flags(p.trunc, tl)};
+      }
+      const uint32_t next = chunk + gridDim.x;
+      have = next < g.nchunks && prefetch(next, slots[buf ^ 1][tid]);
+      buf ^= 1;
+      scan_chunk<Op, BLOCK, LB>(p, g, fd, sm, chunk, tl, f, tid);
+    }
+  }
 }
 
 }  // namespace rlscan

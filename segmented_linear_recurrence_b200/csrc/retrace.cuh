@@ -53,14 +53,15 @@ __device__ __forceinline__ uint32_t load4_flags(const uint8_t *__restrict__ p, u
   return w;
 }
 
-__device__ __forceinline__ void store4(float *__restrict__ p, uint32_t i0, int nvalid, bool vec,
+// Stores the steps whose bit is set in `valid` (bit k: step i0 + k).
+__device__ __forceinline__ void store4(float *__restrict__ p, uint32_t i0, uint32_t valid, bool vec,
                                        const float (&v)[4]) {
-  if (vec && nvalid == 4) {
+  if (vec && valid == 0xfu) {
     __stcs(reinterpret_cast<float4 *>(p + i0), make_float4(v[0], v[1], v[2], v[3]));
   } else {
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-      if (k < nvalid) p[i0 + k] = v[k];
+      if ((valid >> k) & 1u) p[i0 + k] = v[k];
   }
 }
 
@@ -103,7 +104,6 @@ struct RetraceOp {
   struct Nbr {
     float e, qa, c;
   };
-  struct Aux {};
 
   // Dynamic shared memory layout for a chunk of L steps:
   //   float E[L + 1], Qa[L + 1], C[L + 1]   (index L: first step after the chunk)
@@ -132,23 +132,22 @@ struct RetraceOp {
     return Nbr{sE[local], sE[(L + 1) + local], sE[2 * (L + 1) + local]};
   }
 
-  static __device__ __forceinline__ Aff<float> coef(const Args &p, const Item &it, const Nbr &nx,
-                                                    bool row_end, uint32_t n, uint32_t i, Aux &) {
-    bool cont;
-    float nv = successor_value(it.fl, row_end, 0.0f, p.tv, p.boot, n, i, cont);
+  // `cont`, `nv`: from successor_value() (loaded ahead of the staging).
+  static __device__ __forceinline__ Aff<float> coef(const Args &p, const Item &it, const Nbr &nx, bool cont,
+                                                    float nv) {
     if (cont) return Aff<float>{p.gamma * nx.c, fmaf(p.gamma, fmaf(-nx.c, nx.qa, nx.e), it.r)};
     return Aff<float>{0.0f, fmaf(p.gamma, nv, it.r)};
   }
 
-  static __device__ __forceinline__ void emit(const Args &p, uint32_t i0, int nv, bool vec,
-                                              const Item (&)[4], const float (&x)[4],
-                                              const float (&)[4], const Aux (&)[4]) {
-    store4(p.out, i0, nv, vec, x);
+  static __device__ __forceinline__ void emit(const Args &p, uint32_t i0, uint32_t valid, bool vec,
+                                              const float (&x)[4]) {
+    store4(p.out, i0, valid, vec, x);
   }
 
-  // E, q_a and c of one step from its staged rows.
+  // E, q_a and c of one step from its staged rows (act, mu: the step's
+  // action and behaviour probability, loaded ahead).
   static __device__ __forceinline__ void reduce_step(const Args &p, const float *qrow,
-                                                     const float *prow, uint32_t step, float &e,
+                                                     const float *prow, int32_t act, float mu, float &e,
                                                      float &qa, float &c) {
     const uint32_t A = p.A;
     float acc = 0.0f;
@@ -163,8 +162,6 @@ struct RetraceOp {
     } else {
       for (uint32_t a = 0; a < A; ++a) acc = fmaf(prow[a], qrow[a], acc);
     }
-    const int32_t act = __ldg(p.act + step);
-    const float mu = __ldg(p.mu + step);
     float qv = 0.0f, pv = 0.0f;
     if (act >= 0 && uint32_t(act) < A) {
       qv = qrow[act];
@@ -177,11 +174,14 @@ struct RetraceOp {
     c = p.lambda * fminf(1.0f, pv / mu);
   }
 
-  // Fill E / Qa / C for the chunk's steps [cbase, cbase + Lc) and the first
-  // step after it (if any).  Ends with a block barrier.
-  static __device__ void prologue(const Args &p, uint32_t cbase, uint32_t L, uint32_t total,
-                                  unsigned char *smem, int tid, int nthreads,
-                                  uint64_t timeout_ns) {
+  // Fill E / Qa / C for the staged steps [cbase, cbase + Lc) (Lc <= L, cbase
+  // a multiple of 4) and, if `with_next`, for the first step after them.
+  // Ends with a block barrier.  `before_wait()` runs once every copy and load
+  // of the prologue is in flight, before its first wait.
+  template <class Hook>
+  static __device__ void prologue(const Args &p, uint32_t cbase, uint32_t Lc, uint32_t L, bool with_next,
+                                  unsigned char *smem, int tid, int nthreads, uint64_t timeout_ns,
+                                  Hook before_wait) {
     float *sE = reinterpret_cast<float *>(smem);
     float *sQ = sE + (L + 1);
     float *sC = sQ + (L + 1);
@@ -189,10 +189,23 @@ struct RetraceOp {
     float *ring = reinterpret_cast<float *>(smem + scalars_bytes(L));
     const uint32_t stage_floats = 2u * S * A;
     uint64_t *bars = reinterpret_cast<uint64_t *>(ring + NS * stage_floats);
-    const uint32_t Lc = min(L, total - cbase);
     const uint32_t nsub = (Lc + S - 1u) / S;
     const bool use_tma = p.tma != 0u;
     auto full = [&](uint32_t j) { return (j + 1u) * S <= Lc; };
+
+    // Action and behaviour probability of the steps this thread reduces in
+    // the first kAhead sub-tiles: loaded before any wait, so their latency
+    // hides behind the staging copies.
+    constexpr uint32_t kAhead = 4;
+    int32_t act_ahead[kAhead];
+    float mu_ahead[kAhead];
+#pragma unroll
+    for (uint32_t j = 0; j < kAhead; ++j) {
+      const uint32_t local = j * S + uint32_t(tid);
+      const bool mine = j < nsub && uint32_t(tid) < S && local < Lc;
+      act_ahead[j] = mine ? __ldg(p.act + cbase + local) : 0;
+      mu_ahead[j] = mine ? __ldg(p.mu + cbase + local) : 1.0f;
+    }
 
     if (use_tma) {
       if (tid == 0) {
@@ -215,7 +228,7 @@ struct RetraceOp {
 
     // The step after the chunk (its E, q_a, c feed the chunk's last step):
     // one warp reduces it straight from global memory.
-    if (tid < 32 && cbase + Lc < total) {
+    if (tid < 32 && with_next) {
       const uint32_t step = cbase + Lc;
       const size_t off = size_t(step) * A;
       float part = 0.0f;
@@ -238,6 +251,7 @@ struct RetraceOp {
       }
     }
 
+    before_wait();
     for (uint32_t j = 0; j < nsub; ++j) {
       const uint32_t stage = j % NS;
       float *sq = ring + stage * stage_floats;
@@ -255,8 +269,24 @@ struct RetraceOp {
       }
       if (uint32_t(tid) < nst) {
         const uint32_t local = j * S + tid;
+        int32_t act;
+        float mu;
+        if (j < kAhead) {
+          // select from the registers without dynamic indexing
+          act = act_ahead[0];
+          mu = mu_ahead[0];
+#pragma unroll
+          for (uint32_t jj = 1; jj < kAhead; ++jj)
+            if (j == jj) {
+              act = act_ahead[jj];
+              mu = mu_ahead[jj];
+            }
+        } else {
+          act = __ldg(p.act + cbase + local);
+          mu = __ldg(p.mu + cbase + local);
+        }
         float e, qa, c;
-        reduce_step(p, sq + tid * A, sp + tid * A, cbase + local, e, qa, c);
+        reduce_step(p, sq + tid * A, sp + tid * A, act, mu, e, qa, c);
         sE[local] = e;
         sQ[local] = qa;
         sC[local] = c;
@@ -275,18 +305,22 @@ struct RetraceOp {
   }
 };
 
-// One block per chunk of L = 4 * BLOCK steps: the prologue fills E, q_a, c
-// for the chunk (and the step after it) in shared memory, then each thread
-// scans 4 consecutive steps; warps and blocks combine as in scan_kernel.cuh.
-// With LB, blocks take tickets in dependency order (one per block) and chain
-// carries with the decoupled look-back.
+// One block per chunk: the prologue fills E, q_a, c for the chunk's steps
+// (and, with look-back, the step after them) in shared memory, then each
+// thread scans 4 consecutive steps; warps and blocks combine as in
+// scan_kernel.cuh.  Two plans, as there:
+//   LB == false: block b owns the whole rows of the steps [b span, (b + 1)
+//     span); its tiles (and the staging) start at that range's first step
+//     rounded down to a multiple of 4, and steps outside the range are
+//     neither scanned nor stored.
+//   LB == true: chunks of L = 4 * BLOCK steps of the flat sequence, taken in
+//     dependency order by ticket, chained by the decoupled look-back.
 template <int BLOCK, bool LB>
 __global__ void __launch_bounds__(BLOCK) retrace_kernel(const RetraceOp::Args p, const ScanGeom g) {
   using Op = RetraceOp;
   using V = float;
   using Item = Op::Item;
   using Nbr = Op::Nbr;
-  using Aux = Op::Aux;
   constexpr int W = BLOCK / 32;
   constexpr uint32_t L = 4u * BLOCK;
   __shared__ Aff<V> s_wagg[W];
@@ -306,36 +340,56 @@ __global__ void __launch_bounds__(BLOCK) retrace_kernel(const RetraceOp::Args p,
     if (ticket >= g.nchunks) return;  // counter left inconsistent by an aborted launch
     chunk = g.nchunks - 1u - ticket;
   }
-  const uint32_t cbase = chunk * L;
-  Op::prologue(p, cbase, L, g.total, dyn_smem, tid, BLOCK, g.lb.timeout_ns);
+  uint32_t lo, hi, base;
+  if constexpr (LB) {
+    lo = chunk * L;
+    hi = min(lo + L, g.total);
+    base = lo;
+  } else {
+    lo = chunk * g.span;
+    hi = min(lo + g.span, g.total);
+    base = lo & ~3u;
+  }
 
-  const uint32_t i0 = cbase + 4u * uint32_t(tid);
+  // The thread's own steps first: their loads are in flight while the
+  // prologue stages and reduces the chunk's action rows.
+  const uint32_t i0 = base + 4u * uint32_t(tid);
   const int nvalid = i0 < g.total ? int(min(4u, g.total - i0)) : 0;
+  uint32_t valid = i0 < hi ? (1u << min(4u, hi - i0)) - 1u : 0u;
+  if (i0 < lo) valid &= ~((1u << (lo - i0)) - 1u);
   uint32_t n = 0, t = 0;
-  if (nvalid) {
+  if (valid) {
     n = fd.div(i0);
     t = i0 - n * g.T;
   }
   Item it[4];
   Op::load(p, i0, nvalid, g.vec != 0u, it);
+  // Successor values of the thread's boundary steps (trunc_value, bootstrap):
+  // fetched while the staging copies are in flight.
+  bool cont[4];
+  float nvb[4];
+  Op::prologue(p, base, hi - base, L, LB && hi < g.total, dyn_smem, tid, BLOCK, g.lb.timeout_ns, [&] {
+    uint32_t tt = t, nn = n;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      nvb[k] = 0.0f;
+      cont[k] = false;
+      if ((valid >> k) & 1u)
+        nvb[k] = successor_value(it[k].fl, tt == g.T - 1u, 0.0f, p.tv, p.boot, nn, i0 + k, cont[k]);
+      if (++tt == g.T) {
+        tt = 0;
+        ++nn;
+      }
+    }
+  });
   grid_dependents_launch();
   Nbr nb[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) nb[k] = Op::nbr_smem(dyn_smem, L, 4u * uint32_t(tid) + k + 1u);
 
   Aff<V> c[4];
-  Aux aux[4] = {};
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    if (k < nvalid)
-      c[k] = Op::coef(p, it[k], nb[k], t == g.T - 1u, n, i0 + k, aux[k]);
-    else
-      c[k] = aff_identity<V>();
-    if (++t == g.T) {
-      t = 0;
-      ++n;
-    }
-  }
+  for (int k = 0; k < 4; ++k) c[k] = ((valid >> k) & 1u) ? Op::coef(p, it[k], nb[k], cont[k], nvb[k]) : aff_identity<V>();
   Aff<V> agg = compose(c[2], c[3]);
   agg = compose(c[1], agg);
   agg = compose(c[0], agg);
@@ -352,7 +406,7 @@ __global__ void __launch_bounds__(BLOCK) retrace_kernel(const RetraceOp::Args p,
     if constexpr (LB) {
       const V ca = __shfl_sync(0xffffffffu, winc.a, 0);
       const V cb = __shfl_sync(0xffffffffu, winc.b, 0);
-      const bool edge_closed = (min(cbase + L, g.total) % g.T) == 0u;
+      const bool edge_closed = (hi % g.T) == 0u;
       carry = decoupled_lookback<true, V>(g.lb, chunk, g.nchunks, epoch, ticket, Aff<V>{ca, cb}, edge_closed,
                                           lane);
     }
@@ -361,14 +415,13 @@ __global__ void __launch_bounds__(BLOCK) retrace_kernel(const RetraceOp::Args p,
   __syncthreads();
 
   V x = apply(exc, s_wcarry[warp]);
-  V xs[4], xd[4];
+  V xs[4];
 #pragma unroll
   for (int k = 3; k >= 0; --k) {
-    xd[k] = x;
     x = apply(c[k], x);
     xs[k] = x;
   }
-  Op::emit(p, i0, nvalid, g.vec != 0u, it, xs, xd, aux);
+  Op::emit(p, i0, valid, g.vec != 0u, xs);
 }
 
 }  // namespace rlscan

@@ -226,14 +226,14 @@ uint32_t blocks_in_launch(const Plan &pl, int64_t rows, int64_t T) {
 constexpr int kBlocks[] = {128, 192, 256, 320, 384, 448, 512};
 bool valid_block(int64_t b) { return b >= 128 && b <= 512 && b % 64 == 0; }
 
-// Rows plan: the most whole rows of T steps a block of `block` threads can
-// own, whatever the alignment of its first step (0 if one row does not fit).
-// k rows span k T steps, whose 8-step tiles number k T / 8 when k T is a
-// multiple of 8 (every block then starts aligned) and at most
-// (k T + 14) / 8 otherwise.
-int64_t rows_per_block(int64_t T, int block) {
-  auto tiles = [T](int64_t k) { return (k * T) % kTile == 0 ? k * T / kTile : (k * T + 2 * kTile - 2) / kTile; };
-  int64_t k = int64_t(kTile) * block / T;
+// Rows plan: the most whole rows of T steps a block of `block` threads, each
+// scanning a tile of `tile` steps, can own whatever the alignment of its
+// first step (0 if one row does not fit).  k rows span k T steps, whose tiles
+// number k T / tile when k T is a multiple of the tile (every block then
+// starts aligned) and at most (k T + 2 tile - 2) / tile otherwise.
+int64_t rows_per_block(int64_t T, int block, int64_t tile = kTile) {
+  auto tiles = [T, tile](int64_t k) { return (k * T) % tile == 0 ? k * T / tile : (k * T + 2 * tile - 2) / tile; };
+  int64_t k = tile * block / T;
   while (k > 0 && tiles(k) > block) --k;
   return k;
 }
@@ -243,9 +243,30 @@ Plan make_plan(rlscan_estimator est, int64_t N, int64_t T, int64_t A) {
   const int64_t fb = g_force_block.load();
   const bool force_lb = g_force_lookback.load() != 0;
   if (est == RLSCAN_EST_RETRACE) {
-    pl.block = (fb == 128 || fb == 256) ? int(fb) : 128;
-    pl.L = 4u * uint32_t(pl.block);
-    pl.lookback = force_lb || (int64_t(pl.L) % T) != 0;
+    // 4-step tiles, 128- or 256-thread blocks.  Rows plan where a row fits
+    // (the block the rows fill best, the smaller on a tie); else chunks of
+    // 1024 steps with look-back, whose longer chunks halve the chains.
+    int64_t best_k = 0;
+    int best_b = 128;
+    double best_fill = 0.0;
+    for (int b : {128, 256}) {
+      if ((fb == 128 || fb == 256) && b != fb) continue;
+      const int64_t k = rows_per_block(T, b, 4);
+      const double fill = double(k * T) / double(4 * b);
+      if (k > 0 && fill > best_fill + 1e-9) {
+        best_fill = fill;
+        best_k = k;
+        best_b = b;
+      }
+    }
+    pl.lookback = force_lb || best_k == 0;
+    pl.block = (fb == 128 || fb == 256) ? int(fb) : (best_k == 0 ? 256 : best_b);
+    if (pl.lookback) {
+      pl.L = 4u * uint32_t(pl.block);
+    } else {
+      pl.rows_per_block = best_k;
+      pl.L = uint32_t(best_k * T);
+    }
   } else {
     // Rows plan where a row fits a block: the block size whose threads the
     // rows fill best (the smaller one on a tie); else the look-back plan.
@@ -280,16 +301,18 @@ Plan make_plan(rlscan_estimator est, int64_t N, int64_t T, int64_t A) {
   }
   pl.ws_bytes = sizeof(LookbackHeader) + (pl.lookback ? size_t(pl.max_chunks) * sizeof(LookbackDesc) : 0);
   if (est == RLSCAN_EST_RETRACE) {
-    // Sub-tile steps and ring depth: the largest staging that keeps at least
-    // three blocks resident per SM (<= ~72 KB of shared memory each).
-    const uint32_t budget = 72u * 1024u;
+    // Sub-tile steps and ring depth: the largest staging within ~56 KB of
+    // shared memory per block (four blocks per SM), the size that measured
+    // fastest.  The layout is sized for a full chunk of 4 * block steps.
+    const uint32_t budget = 56u * 1024u;
+    const uint32_t Lmax = 4u * uint32_t(pl.block);
     uint32_t S = uint32_t(pl.block);
     uint32_t NS = 4;
-    while (NS > 2 && RetraceOp::smem_bytes(pl.L, S, uint32_t(A), NS) > budget) --NS;
-    while (S > 4 && RetraceOp::smem_bytes(pl.L, S, uint32_t(A), NS) > budget) S = std::max(4u, (S / 2) & ~3u);
+    while (NS > 2 && RetraceOp::smem_bytes(Lmax, S, uint32_t(A), NS) > budget) --NS;
+    while (S > 4 && RetraceOp::smem_bytes(Lmax, S, uint32_t(A), NS) > budget) S = std::max(4u, (S / 2) & ~3u);
     pl.sub_steps = S;
     pl.stages = NS;
-    pl.smem = RetraceOp::smem_bytes(pl.L, S, uint32_t(A), NS);
+    pl.smem = RetraceOp::smem_bytes(Lmax, S, uint32_t(A), NS);
   }
   return pl;
 }

@@ -102,7 +102,7 @@ def load_traffic(kernel_key: str):
     if j.get("source_hash") != slr_build.source_hash():
         return None
     k = j.get("kernels", {}).get(kernel_key)
-    return None if k is None else k.get("dram_bytes_per_full_launch")
+    return None if k is None else k.get("dram_bytes_per_launch")
 
 
 # ---------------------------------------------------------------------------
@@ -446,6 +446,27 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+def run_one(args):
+    """`--one EST N T [A]`: `--steps` plain calls of one estimator on seeded
+    inputs of the workload recipe (p_term 0.02, p_trunc 0.005 where the
+    estimator takes truncation), for ncu captures of a single kernel."""
+    import torch
+    import segmented_linear_recurrence_b200 as slr
+    from segmented_linear_recurrence_b200 import build as slr_build
+    slr_build.build()
+    est, N, T = args.one[0], int(args.one[1]), int(args.one[2])
+    A = int(args.one[3]) if len(args.one) > 3 else 18
+    trunc = 0.0 if est in ("retrace", "elig_trace", "episodic_prefix_sum") else 0.005
+    d = synthetic.make_inputs(est, N, T, seed=5, p_term=0.02, p_trunc=trunc, A=A, with_init=True)
+    call = DeviceCall(est, T, d, torch.device("cuda", 0))
+    for _ in range(max(args.steps, 1)):
+        call.launch()
+    torch.cuda.synchronize()
+    st = slr.rlscan_sync_status()
+    print(json.dumps({"one": est, "N": N, "T": T, "A": A, "calls": args.steps, "status": st}))
+    return 0 if st == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -456,10 +477,14 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU work for the oracle baseline (0 disables it)")
+    ap.add_argument("--one", nargs="+", metavar="EST N T [A]",
+                    help="only run --steps plain calls of one estimator (for profiling)")
     args = ap.parse_args()
 
     if args.impl == "reference":
         return run_reference(args)
+    if args.one:
+        return run_one(args)
 
     import torch
     import torch.distributed as dist

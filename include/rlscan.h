@@ -47,13 +47,15 @@
  * Scalars.  gamma, lambda, rho_bar, c_bar must be finite; rho_bar, c_bar > 0.
  * Streams.  Every call is asynchronous on `stream` (NULL = legacy default
  *   stream).  Calls on different streams may run concurrently.
- * Scratch.  Thread blocks draw chunks of work from a ticket counter, and long
- *   rows (more steps than one chunk) are split across chunks that hand their
- *   carries to one another; both live in a small per-(device, stream)
- *   workspace the library allocates on the first call on that stream and
- *   keeps until rlscan_release_workspaces().  Allocation is not allowed while
- *   `stream` is being captured into a CUDA graph: make one call of the same or
- *   larger size on that stream before capturing.
+ * Scratch.  Rows that fit one thread block (up to about 4096 steps; Retrace
+ *   512 or 1024) need none: each block owns whole rows.  Longer rows are
+ *   split into chunks that thread blocks draw from a ticket counter and that
+ *   hand their carries to one another; counter and carries live in a small
+ *   per-(device, stream) workspace the library allocates on the first such
+ *   call on that stream and keeps until rlscan_release_workspaces().
+ *   Allocation is not allowed while `stream` is being captured into a CUDA
+ *   graph: make one call of the same or larger size on that stream (or call
+ *   rlscan_reserve_workspace) before capturing.
  * Errors.  Invalid arguments are reported synchronously and launch nothing.
  *   Conditions only the device can see (a carry hand-off that timed out, an
  *   action index outside [0, A)) are recorded in a per-device status word
@@ -255,8 +257,9 @@ typedef struct rlscan_plan_info {
   int32_t chunk_steps;      /* steps one thread block scans */
   int32_t lookback;         /* 1: blocks chain their carries through the workspace */
   int32_t launches;         /* kernel launches the call makes (row slices) */
-  int64_t chunks;           /* chunks of chunk_steps steps over all launches; persistent
-                               blocks draw them from a ticket counter */
+  int64_t chunks;           /* chunks over all launches: groups of whole rows (walked by
+                               resident blocks) or, with look-back, pieces of
+                               chunk_steps steps drawn by ticket */
   int64_t workspace_bytes;  /* workspace the call needs on its stream */
 } rlscan_plan_info;
 

@@ -29,9 +29,10 @@ NVCC_FLAGS = [
 
 
 def source_hash() -> str:
-    """Hash of every kernel source and the build flags (identifies a kernel build)."""
+    """Hash of every kernel source (csrc/) and the build flags: identifies the
+    kernels a profile was taken on (the public header's comments do not)."""
     h = hashlib.sha256()
-    for path in sorted(DEPS):
+    for path in sorted(d for d in DEPS if os.path.dirname(d) == CSRC):
         h.update(os.path.basename(path).encode())
         with open(path, "rb") as f:
             h.update(f.read())

@@ -79,10 +79,13 @@ __device__ __forceinline__ void ld8(const int32_t *p, const Tile &tl, uint32_t (
   }
 }
 
-// Bit k set iff byte k of the 8 bytes is nonzero.
+// Bit j set iff byte j of the word is nonzero.  Per byte x, (x & 0x7f) + 0x7f
+// carries into bit 7 iff x & 0x7f != 0 and never out of the byte; or-ing x
+// adds x's own bit 7.  The multiply then moves bits 7, 15, 23, 31 to 28..31
+// (shifts of 21, 14, 7, 0; no two partial products share a bit).
 __device__ __forceinline__ uint32_t nonzero_bytes4(uint32_t w) {
-  const uint32_t ones = __vcmpne4(w, 0u) & 0x01010101u;  // bit 8j set iff byte j != 0
-  return ((ones * 0x00204081u) >> 21) & 0xfu;             // gather bits 0, 8, 16, 24
+  const uint32_t hi = (((w & 0x7f7f7f7fu) + 0x7f7f7f7fu) | w) & 0x80808080u;
+  return (hi * 0x00204081u) >> 28;
 }
 __device__ __forceinline__ uint32_t ld8_flags(const uint8_t *p, const Tile &tl) {
   if (p == nullptr) return 0u;
@@ -136,26 +139,27 @@ struct Flags {
   uint32_t term, trunc;
 };
 
-// trunc_value at the tile's truncated (not terminated) steps: the only loads
-// whose addresses depend on loaded data.  Warps without such a step skip them.
-__device__ __forceinline__ void trunc_values(const float *tv, const Tile &tl, Flags f, float (&sv)[8]) {
+// Successor values of the tile's boundary steps (backward estimators), 0 at
+// every other step: 0 after termination, trunc_value after truncation, the
+// row's bootstrap at a row end (`boot` may be NULL: 0); termination wins over
+// truncation, and both over the row end.  trunc_value is the only load whose
+// address depends on loaded data; warps without a truncated step skip it.
+__device__ __forceinline__ void boundary_successors(const float *tv, const float *boot, float ev, const Tile &tl,
+                                                    Flags f, const FastDiv &fd, float (&bv)[8]) {
   const uint32_t tr = f.trunc & ~f.term & tl.valid;
+  const uint32_t ed = tl.edge & ~f.term & ~f.trunc;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) sv[k] = 0.0f;
-  if (!__any_sync(0xffffffffu, tr != 0u)) return;
+  for (int k = 0; k < 8; ++k) bv[k] = 0.0f;
+  if (__any_sync(0xffffffffu, tr != 0u)) {
 #pragma unroll
-  for (int k = 0; k < 8; ++k)
-    if ((tr >> k) & 1u) sv[k] = __ldg(tv + tl.i0 + k);
-}
-
-// Successor value of boundary step k (backward estimators): 0 after
-// termination, trunc_value after truncation, the row's bootstrap at a row end
-// (`boot` may be NULL: 0).
-__device__ __forceinline__ float boundary_value(int k, Flags f, const float (&sv)[8], float ev, const float *boot,
-                                                const Tile &tl, const FastDiv &fd) {
-  if ((f.term >> k) & 1u) return 0.0f;
-  if ((f.trunc >> k) & 1u) return sv[k];
-  return tl.few_rows ? ev : (boot ? __ldg(boot + tl.n0 + fd.div(tl.t0 + k)) : 0.0f);
+    for (int k = 0; k < 8; ++k)
+      if ((tr >> k) & 1u) bv[k] = __ldg(tv + tl.i0 + k);
+  }
+  if (ed != 0u) {  // at most one row end per tile when T >= 8
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if ((ed >> k) & 1u) bv[k] = tl.few_rows ? ev : (boot ? __ldg(boot + tl.n0 + fd.div(tl.t0 + k)) : 0.0f);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -173,7 +177,7 @@ struct GaeOp {
     float gamma, gl;
   };
   struct Raw {
-    float r[8], v[8], sv[8];  // sv: trunc_value at truncated steps
+    float r[8], v[8], bv[8];  // bv: successor values at boundary steps
     Flags f;
     float halo;  // v of the step after the tile (lane 31 only)
     float ev;    // bootstrap of the tile's row end
@@ -186,8 +190,8 @@ struct GaeOp {
     w.halo = (lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total) ? __ldg(p.v + tl.i0 + 8u) : 0.0f;
     w.ev = edge_value(p.boot, tl, fd);
   }
-  static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, Raw &w) {
-    trunc_values(p.tv, tl, w.f, w.sv);
+  static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w) {
+    boundary_successors(p.tv, p.boot, w.ev, tl, w.f, fd, w.bv);
   }
   static __device__ __forceinline__ float nbr_of(const Raw &w) { return w.v[0]; }
   static __device__ __forceinline__ float halo_of(const Raw &w) { return w.halo; }
@@ -198,7 +202,7 @@ struct GaeOp {
     for (int k = 0; k < 8; ++k) {
       const bool sp = (special >> k) & 1u;
       const float next = k < 7 ? w.v[k < 7 ? k + 1 : 7] : next7;
-      const float nv = sp ? boundary_value(k, w.f, w.sv, w.ev, p.boot, tl, fd) : next;
+      const float nv = sp ? w.bv[k] : next;
       c[k] = Aff<float>{sp ? 0.0f : p.gl, fmaf(p.gamma, nv, w.r[k]) - w.v[k]};
     }
   }
@@ -229,7 +233,7 @@ struct TdLambdaOp {
     float gamma, gl, g1l;  // gamma, gamma*lambda, gamma*(1-lambda)
   };
   struct Raw {
-    float r[8], v[8], sv[8];
+    float r[8], v[8], bv[8];
     Flags f;
     float halo, ev;
   };
@@ -241,8 +245,8 @@ struct TdLambdaOp {
     w.halo = (lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total) ? __ldg(p.v + tl.i0 + 8u) : 0.0f;
     w.ev = edge_value(p.boot, tl, fd);
   }
-  static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, Raw &w) {
-    trunc_values(p.tv, tl, w.f, w.sv);
+  static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w) {
+    boundary_successors(p.tv, p.boot, w.ev, tl, w.f, fd, w.bv);
   }
   static __device__ __forceinline__ float nbr_of(const Raw &w) { return w.v[0]; }
   static __device__ __forceinline__ float halo_of(const Raw &w) { return w.halo; }
@@ -253,8 +257,7 @@ struct TdLambdaOp {
     for (int k = 0; k < 8; ++k) {
       const bool sp = (special >> k) & 1u;
       const float next = k < 7 ? w.v[k < 7 ? k + 1 : 7] : next7;
-      c[k] = sp ? Aff<float>{0.0f, fmaf(p.gamma, boundary_value(k, w.f, w.sv, w.ev, p.boot, tl, fd), w.r[k])}
-                : Aff<float>{p.gl, fmaf(p.g1l, next, w.r[k])};
+      c[k] = sp ? Aff<float>{0.0f, fmaf(p.gamma, w.bv[k], w.r[k])} : Aff<float>{p.gl, fmaf(p.g1l, next, w.r[k])};
     }
   }
   static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[8],
@@ -278,7 +281,7 @@ struct DiscountedOp {
     float gamma;
   };
   struct Raw {
-    float r[8], sv[8];
+    float r[8], bv[8];
     Flags f;
     float ev;
   };
@@ -288,8 +291,8 @@ struct DiscountedOp {
     w.f = f;
     w.ev = edge_value(p.boot, tl, fd);
   }
-  static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, Raw &w) {
-    trunc_values(p.tv, tl, w.f, w.sv);
+  static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w) {
+    boundary_successors(p.tv, p.boot, w.ev, tl, w.f, fd, w.bv);
   }
   static __device__ __forceinline__ float nbr_of(const Raw &) { return 0.0f; }
   static __device__ __forceinline__ float halo_of(const Raw &) { return 0.0f; }
@@ -299,8 +302,7 @@ struct DiscountedOp {
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const bool sp = (special >> k) & 1u;
-      c[k] = sp ? Aff<float>{0.0f, fmaf(p.gamma, boundary_value(k, w.f, w.sv, w.ev, p.boot, tl, fd), w.r[k])}
-                : Aff<float>{p.gamma, w.r[k]};
+      c[k] = Aff<float>{sp ? 0.0f : p.gamma, fmaf(p.gamma, w.bv[k], w.r[k])};
     }
   }
   static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[8],
@@ -327,7 +329,7 @@ struct VtraceOp {
     float gamma, lambda, rho_bar, c_bar;
   };
   struct Raw {
-    float lr[8], r[8], v[8], sv[8];  // coef() keeps gamma * rho * cont in lr for emit()
+    float lr[8], r[8], v[8], bv[8];  // coef() keeps gamma * rho * cont in lr for emit()
     Flags f;
     float halo, ev;
   };
@@ -340,8 +342,8 @@ struct VtraceOp {
     w.halo = (lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total) ? __ldg(p.v + tl.i0 + 8u) : 0.0f;
     w.ev = edge_value(p.boot, tl, fd);
   }
-  static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, Raw &w) {
-    trunc_values(p.tv, tl, w.f, w.sv);
+  static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w) {
+    boundary_successors(p.tv, p.boot, w.ev, tl, w.f, fd, w.bv);
   }
   static __device__ __forceinline__ float nbr_of(const Raw &w) { return w.v[0]; }
   static __device__ __forceinline__ float halo_of(const Raw &w) { return w.halo; }
@@ -352,7 +354,7 @@ struct VtraceOp {
     for (int k = 0; k < 8; ++k) {
       const bool sp = (special >> k) & 1u;
       const float next = k < 7 ? w.v[k < 7 ? k + 1 : 7] : next7;
-      const float nv = sp ? boundary_value(k, w.f, w.sv, w.ev, p.boot, tl, fd) : next;
+      const float nv = sp ? w.bv[k] : next;
       const float ratio = __expf(w.lr[k]);
       const float rho = fminf(p.rho_bar, ratio);
       const float cc = p.lambda * fminf(p.c_bar, ratio);
@@ -404,7 +406,7 @@ struct EligOp {
       w.halo = ((p.term && __ldg(p.term + tl.i0 - 1u)) || (p.trunc && __ldg(p.trunc + tl.i0 - 1u))) ? 1u : 0u;
     w.ev = edge_value(p.init, tl, fd);
   }
-  static __device__ __forceinline__ void fetch_boundary(const Args &, const Tile &, Raw &) {}
+  static __device__ __forceinline__ void fetch_boundary(const Args &, const Tile &, const FastDiv &, Raw &) {}
   static __device__ __forceinline__ uint32_t nbr_of(const Raw &w) { return (w.done >> 7) & 1u; }
   static __device__ __forceinline__ uint32_t halo_of(const Raw &w) { return w.halo; }
   static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w,
@@ -450,7 +452,7 @@ struct PrefixSumOp {
     if (lane == 0 && tl.i0 > 0u && tl.nvalid > 0)
       w.halo = ((p.term && __ldg(p.term + tl.i0 - 1u)) || (p.trunc && __ldg(p.trunc + tl.i0 - 1u))) ? 1u : 0u;
   }
-  static __device__ __forceinline__ void fetch_boundary(const Args &, const Tile &, Raw &) {}
+  static __device__ __forceinline__ void fetch_boundary(const Args &, const Tile &, const FastDiv &, Raw &) {}
   static __device__ __forceinline__ uint32_t nbr_of(const Raw &w) { return (w.done >> 7) & 1u; }
   static __device__ __forceinline__ uint32_t halo_of(const Raw &w) { return w.halo; }
   static __device__ __forceinline__ void coef(const Args &, const Tile &tl, const FastDiv &, Raw &w, uint32_t prev7,

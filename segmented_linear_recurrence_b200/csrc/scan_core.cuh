@@ -71,16 +71,17 @@ __device__ __forceinline__ bool cuts(Aff<uint32_t> f) { return f.a == 0u; }
 
 // Lane l receives the inclusive composite, in dependency order, of the lanes
 // it depends on: BACKWARD lanes l..31 (agg_l o agg_{l+1} o ... o agg_31),
-// forward lanes l..0 (agg_l o agg_{l-1} o ... o agg_0).
-template <bool BACKWARD, typename V>
+// forward lanes l..0 (agg_l o agg_{l-1} o ... o agg_0).  With WIDTH < 32 only
+// lanes 0..WIDTH-1 are scanned (log2 WIDTH rounds).
+template <bool BACKWARD, typename V, int WIDTH = 32>
 __device__ __forceinline__ Aff<V> warp_inclusive_scan(Aff<V> s, int lane) {
 #pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
+  for (int d = 1; d < WIDTH; d <<= 1) {
     V oa, ob;
     if (BACKWARD) {
       oa = __shfl_down_sync(0xffffffffu, s.a, d);
       ob = __shfl_down_sync(0xffffffffu, s.b, d);
-      if (lane + d < 32) s = compose(s, Aff<V>{oa, ob});
+      if (lane + d < WIDTH) s = compose(s, Aff<V>{oa, ob});
     } else {
       oa = __shfl_up_sync(0xffffffffu, s.a, d);
       ob = __shfl_up_sync(0xffffffffu, s.b, d);

@@ -45,7 +45,8 @@ struct ScanGeom {
   uint32_t total;         // steps in this launch (rows * T)
   uint32_t T;             // steps per row
   uint32_t nchunks;       // chunks (blocks) in this launch
-  uint32_t span;          // rows plan: steps per block (k T)
+  uint32_t span;          // rows plan: steps per chunk (k T)
+  uint32_t rows_per_chunk;  // rows plan: k
   uint32_t vec;           // 1: arrays aligned for 256-bit (flags: 64-bit) accesses
   uint32_t div_m, div_l;  // FastDiv by T
   LookbackCtl lb;         // ticket / done / epoch counters and descriptors (look-back only)
@@ -151,6 +152,7 @@ struct ScanSmem {
   static constexpr int W = BLOCK / 32;
   static constexpr int kParked = LB ? int(sizeof(Aff<V>) * kTile / 4) : 1;
   Aff<V> wagg[W];
+  Aff<V> wagg2[2][W];  // rows plan: double-buffered by chunk
   V wcarry[W];
   uint32_t ticket, epoch;
   uint32_t park[kParked][32];
@@ -158,6 +160,32 @@ struct ScanSmem {
 
 // One chunk: the block's steps [lo, hi), tiles from `base`.  `f` holds the
 // thread's flag masks.  Look-back plan: `chunk` is the ticketed chunk.
+// a8: re-sweep the thread's steps from the carry x entering its tile and
+// write the outputs.
+template <class Op>
+__device__ __forceinline__ void resweep_and_emit(const typename Op::Args &p, const Tile &tl,
+                                                 const typename Op::Raw &w,
+                                                 const Aff<typename Op::V> (&c)[kTile], typename Op::V x) {
+  using V = typename Op::V;
+  V xs[kTile], xd[kTile];
+  if (Op::kBackward) {
+#pragma unroll
+    for (int k = kTile - 1; k >= 0; --k) {
+      xd[k] = x;
+      x = apply(c[k], x);
+      xs[k] = x;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < kTile; ++k) {
+      xd[k] = x;
+      x = apply(c[k], x);
+      xs[k] = x;
+    }
+  }
+  Op::emit(p, tl, w, c, xs, xd);
+}
+
 // Rows plan: the loads that depend on the flags go out right behind the
 // tile's other loads (the flags are normally in hand already, prefetched).
 // Look-back plan: they follow once the tile's own loads have arrived, which
@@ -165,7 +193,7 @@ struct ScanSmem {
 template <class Op, int BLOCK, bool LB>
 __device__ __forceinline__ void scan_chunk(const typename Op::Args &p, const ScanGeom &g, const FastDiv &fd,
                                            ScanSmem<Op, BLOCK, LB> &sm, uint32_t chunk, const Tile &tl, Flags f,
-                                           int tid) {
+                                           int tid, int sm_buf) {
   constexpr bool early = !LB;
   using V = typename Op::V;
   using Raw = typename Op::Raw;
@@ -177,7 +205,7 @@ __device__ __forceinline__ void scan_chunk(const typename Op::Args &p, const Sca
   // a1: every load of the tile goes out together.
   Raw w;
   Op::load(p, tl, fd, lane, g.total, f, w);
-  if constexpr (early) Op::fetch_boundary(p, tl, w);
+  if constexpr (early) Op::fetch_boundary(p, tl, fd, w);
   // Every block has issued its loads: the next kernel may start launching.
   grid_dependents_launch();
 
@@ -185,7 +213,7 @@ __device__ __forceinline__ void scan_chunk(const typename Op::Args &p, const Sca
   auto mine = Op::nbr_of(w);
   auto from = BWD ? __shfl_down_sync(0xffffffffu, mine, 1) : __shfl_up_sync(0xffffffffu, mine, 1);
   if (BWD ? lane == 31 : lane == 0) from = Op::halo_of(w);
-  if constexpr (!early) Op::fetch_boundary(p, tl, w);
+  if constexpr (!early) Op::fetch_boundary(p, tl, fd, w);
 
   // a2: coefficients in registers.
   Aff<V> c[kTile];
@@ -211,8 +239,29 @@ __device__ __forceinline__ void scan_chunk(const typename Op::Args &p, const Sca
   // a5: warp scan.
   const Aff<V> inc = warp_inclusive_scan<BWD>(agg, lane);
   const Aff<V> exc = warp_exclusive_from_inclusive<BWD>(inc, lane, 31);
-  if (BWD ? lane == 0 : lane == 31) sm.wagg[warp] = inc;
+  if (BWD ? lane == 0 : lane == 31) {
+    if constexpr (LB)
+      sm.wagg[warp] = inc;
+    else
+      sm.wagg2[sm_buf][warp] = inc;
+  }
   __syncthreads();
+
+  if constexpr (!LB) {
+    // Rows plan: the chunk needs no carry from outside, so every warp scans
+    // the W warp aggregates itself (one barrier per chunk): the carry entering
+    // warp w is the composite of the warps after it (backward) / before it
+    // (forward), applied to 0.  Aggregates alternate between two buffers so
+    // the next chunk's writes never meet this chunk's reads.
+    constexpr int kWidth = W <= 4 ? 4 : (W <= 8 ? 8 : (W <= 16 ? 16 : 32));
+    const Aff<V> wv = lane < W ? sm.wagg2[sm_buf][lane] : aff_identity<V>();
+    const Aff<V> winc = warp_inclusive_scan<BWD, V, kWidth>(wv, lane);
+    const int src = BWD ? warp + 1 : warp - 1;
+    const V nb = __shfl_sync(0xffffffffu, winc.b, src < 0 ? 0 : (src >= W ? W - 1 : src));
+    const V carry_w = (src < 0 || src >= W) ? V(0) : nb;
+    resweep_and_emit<Op>(p, tl, w, c, apply(exc, carry_w));
+    return;
+  }
 
   // a6 (+ a7): warp 0 scans the warp aggregates; with look-back it also
   // obtains the carry entering the chunk.
@@ -236,25 +285,7 @@ __device__ __forceinline__ void scan_chunk(const typename Op::Args &p, const Sca
   }
   __syncthreads();
 
-  // a8: re-sweep the thread's steps from the carry and write the outputs.
-  V x = apply(exc, sm.wcarry[warp]);
-  V xs[kTile], xd[kTile];
-  if (BWD) {
-#pragma unroll
-    for (int k = kTile - 1; k >= 0; --k) {
-      xd[k] = x;
-      x = apply(c[k], x);
-      xs[k] = x;
-    }
-  } else {
-#pragma unroll
-    for (int k = 0; k < kTile; ++k) {
-      xd[k] = x;
-      x = apply(c[k], x);
-      xs[k] = x;
-    }
-  }
-  Op::emit(p, tl, w, c, xs, xd);
+  resweep_and_emit<Op>(p, tl, w, c, apply(exc, sm.wcarry[warp]));
 }
 
 template <class Op, int BLOCK, bool LB>
@@ -283,7 +314,7 @@ __global__ void __launch_bounds__(BLOCK, (min_blocks_per_sm<Op, BLOCK, LB>()))
     const uint32_t lo = chunk * L, hi = min(lo + L, g.total);
     const Tile tl = make_tile<BWD>(g, fd, lo + uint32_t(kTile) * uint32_t(tid), lo, hi);
     const Flags f{ld8_flags(p.term, tl), ld8_flags(p.trunc, tl)};
-    scan_chunk<Op, BLOCK, LB>(p, g, fd, sm, chunk, tl, f, tid);
+    scan_chunk<Op, BLOCK, LB>(p, g, fd, sm, chunk, tl, f, tid, 0);
   } else {
     // Rows plan, persistent: the block takes chunks blockIdx.x, + gridDim.x,
     // ...  While it scans one chunk, its threads prefetch the next chunk's
@@ -306,10 +337,30 @@ __global__ void __launch_bounds__(BLOCK, (min_blocks_per_sm<Op, BLOCK, LB>()))
       asm volatile("cp.async.commit_group;" ::: "memory");
       return true;
     };
+    // When every chunk starts on an 8-step boundary (k T a multiple of 8), a
+    // thread's tile has the same offset, time and row edges in every full
+    // chunk: only its first step and row move.  Holding that tile across the
+    // loop costs registers, so estimators on a 32-register budget (where it
+    // measured slower) rebuild the tile per chunk instead.
+    constexpr bool kKeepTile = Op::kRegs >= 40;
+    const bool aligned = kKeepTile && (g.span % uint32_t(kTile)) == 0u && g.span <= g.total;
+    Tile inv = make_tile<BWD>(g, fd, uint32_t(kTile) * uint32_t(tid), 0u, g.span);
+    if (inv.valid == 0u) {  // thread beyond the chunk's steps: loads nothing
+      inv.nvalid = 0;
+      inv.fast = inv.full = false;
+    }
     bool have = false;  // slots[buf][tid] holds this chunk's flags
     int buf = 0;
     for (uint32_t chunk = blockIdx.x; chunk < g.nchunks; chunk += gridDim.x) {
-      const Tile tl = tile_of(chunk);
+      const uint32_t lo = chunk * g.span;
+      Tile tl;
+      if (aligned && lo + g.span <= g.total) {
+        tl = inv;
+        tl.i0 = lo + uint32_t(kTile) * uint32_t(tid);
+        tl.n0 = inv.n0 + chunk * g.rows_per_chunk;
+      } else {
+        tl = tile_of(chunk);
+      }
       Flags f;
       if (have) {
         asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -321,8 +372,8 @@ __global__ void __launch_bounds__(BLOCK, (min_blocks_per_sm<Op, BLOCK, LB>()))
       }
       const uint32_t next = chunk + gridDim.x;
       have = next < g.nchunks && prefetch(next, slots[buf ^ 1][tid]);
+      scan_chunk<Op, BLOCK, LB>(p, g, fd, sm, chunk, tl, f, tid, buf);
       buf ^= 1;
-      scan_chunk<Op, BLOCK, LB>(p, g, fd, sm, chunk, tl, f, tid);
     }
   }
 }

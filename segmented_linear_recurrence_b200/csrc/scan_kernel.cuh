@@ -135,9 +135,12 @@ constexpr int min_blocks_per_sm() {
 // Flag bytes of one tile, prefetched into shared memory for the block's next
 // chunk: each thread copies its own tile's 8 terminated and 8 truncated bytes
 // with cp.async and reads them back itself (no barrier needed).
-struct FlagSlot {
+// 16-byte aligned: the 8-byte cp.async copies need an 8-byte aligned
+// destination, whatever the shared-memory layout around the slots.
+struct __align__(16) FlagSlot {
   uint32_t term[2], trunc[2];
 };
+static_assert(alignof(FlagSlot) >= 8 && sizeof(FlagSlot) == 16, "cp.async destinations must stay aligned");
 
 __device__ __forceinline__ void cp_async8(void *dst_smem, const void *src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst_smem))),

@@ -11,6 +11,7 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <type_traits>
 #include <utility>
 #include <vector>
@@ -330,18 +331,18 @@ void fast_div_params(uint32_t d, uint32_t &m, uint32_t &l) {
 }
 
 // Blocks of `kern` that fit on the current device at once (occupancy x SMs),
-// cached per (device, kernel).
-int resident_blocks(const void *kern, int block) {
+// cached per (device, kernel, dynamic shared size).
+int resident_blocks(const void *kern, int block, size_t dyn_smem = 0) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 1;
   static std::mutex mu;
-  static std::map<std::pair<int, const void *>, int> cache;
+  static std::map<std::tuple<int, const void *, size_t>, int> cache;
   std::lock_guard<std::mutex> lock(mu);
-  const auto key = std::make_pair(dev, kern);
+  const auto key = std::make_tuple(dev, kern, dyn_smem);
   const auto it = cache.find(key);
   if (it != cache.end()) return it->second;
   int per_sm = 0, sms = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, block, 0) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, block, dyn_smem) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
     cudaGetLastError();
     return 1;

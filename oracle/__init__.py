@@ -1,7 +1,8 @@
-"""fp64 CPU oracle for the seven estimators -- TEST INFRASTRUCTURE ONLY.
+"""fp64 CPU oracle for the seven estimators and the generic affine scan -- TEST
+INFRASTRUCTURE ONLY.
 
 Only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline / reference
 leg may import anything from this package.  The product library never does.
 """
-from .oracle import (discounted_return, elig_trace, episodic_prefix_sum, gae, retrace,  # noqa: F401
-                     run, td_lambda, vtrace)
+from .oracle import (affine_scan, discounted_return, elig_trace, episodic_prefix_sum, gae,  # noqa: F401
+                     retrace, run, td_lambda, vtrace)

@@ -33,6 +33,7 @@ def bind(lib):
         "rlo_retrace": [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, dbl, dbl, vp],
         "rlo_elig_trace": [i64, i64, vp, vp, vp, vp, dbl, dbl, vp],
         "rlo_episodic_prefix_sum": [i64, i64, vp, vp, vp, vp, vp],
+        "rlo_affine_scan": [i64, i64, vp, vp, vp, vp, ctypes.c_int, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -160,12 +161,24 @@ def episodic_prefix_sum(x, terminated, truncated=None):
     return out, int(mx.value)
 
 
+def affine_scan(a, b, reset=None, init=None, reverse=False):
+    """x_t = b_t + a_t x_prev in scan order (backward when `reverse`), x_prev
+    = init[n] (None: 0) at the row's first step, x_t = b_t where reset."""
+    N, T = _dims(a)
+    keep = [_p(a, np.float32), _p(b, np.float32), _p(reset, np.uint8), _p(init, np.float32)]
+    out = np.empty((N, T), np.float64)
+    rc = _load().rlo_affine_scan(N, T, *[k[1] for k in keep], 1 if reverse else 0,
+                                 out.ctypes.data_as(ctypes.c_void_p))
+    _check(rc, "affine_scan")
+    return out
+
+
 # Convenience: dispatch by estimator name on a dict of inputs as produced by
 # segmented_linear_recurrence_b200.synthetic (keys match parameter names).
 def run(name, inp, **scal):
     fn = {"gae": gae, "td_lambda": td_lambda, "discounted_return": discounted_return,
           "vtrace": vtrace, "retrace": retrace, "elig_trace": elig_trace,
-          "episodic_prefix_sum": episodic_prefix_sum}[name]
+          "episodic_prefix_sum": episodic_prefix_sum, "affine_scan": affine_scan}[name]
     params = inspect.signature(fn).parameters
     kw = {k: v for k, v in inp.items() if k in params}
     kw.update({k: v for k, v in scal.items() if k in params})
@@ -173,4 +186,4 @@ def run(name, inp, **scal):
 
 
 __all__ = ["gae", "td_lambda", "discounted_return", "vtrace", "retrace", "elig_trace",
-           "episodic_prefix_sum", "run"]
+           "episodic_prefix_sum", "affine_scan", "run"]

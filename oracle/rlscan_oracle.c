@@ -291,3 +291,28 @@ int rlo_episodic_prefix_sum(int64_t N, int64_t T, const int32_t *x,
   if (max_abs) *max_abs = m;
   return 0;
 }
+
+/* Generic first-order linear recurrence (the pages' unified form, gist.science
+ * technical summary, Methodologie 1, with the coefficients given directly):
+ * in scan order (t = 0..T-1 forward, t = T-1..0 when `reverse`),
+ *   x_t = b_t + a_t * x_prev,
+ * where x_prev is the previous step in scan order, or init[n] (NULL: 0) for
+ * the row's first step; reset[t] != 0 (reset may be NULL) cuts the
+ * dependency, x_t = b_t. */
+int rlo_affine_scan(int64_t N, int64_t T, const float *a, const float *b,
+                    const uint8_t *reset, const float *init, int reverse,
+                    double *x) {
+  if (bad_dims(N, T)) return -1;
+  for (int64_t n = 0; n < N; ++n) {
+    double carry = init ? (double)init[n] : 0.0;
+    for (int64_t k = 0; k < T; ++k) {
+      const int64_t t = reverse ? T - 1 - k : k;
+      const int64_t i = n * T + t;
+      double v = (double)b[i];
+      if (!(reset && reset[i])) v += (double)a[i] * carry;
+      x[i] = v;
+      carry = v;
+    }
+  }
+  return 0;
+}

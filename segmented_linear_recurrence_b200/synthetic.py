@@ -121,3 +121,16 @@ def workload_inputs(workload: str, estimator: str, T: int | None = None) -> dict
 
 def input_bytes(d: dict) -> int:
     return int(sum(v.nbytes for v in d.values() if isinstance(v, np.ndarray)))
+
+
+def make_affine_inputs(N: int, T: int, *, seed: int, p_reset: float = 0.01, with_init: bool = True,
+                       a_low: float = 0.8, a_high: float = 1.0) -> dict:
+    """Seeded inputs of the generic affine scan: a ~ U(a_low, a_high) (decay
+    factors such as gamma * lambda), b ~ N(0, 1), reset ~ Bernoulli(p_reset)
+    (uint8, None when p_reset is 0), init ~ N(0, 1) per row (or None)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    a = rng.uniform(a_low, a_high, size=(N, T)).astype(np.float32)
+    b = _normal(rng, (N, T))
+    reset = (rng.random((N, T)) < p_reset).astype(np.uint8) if p_reset > 0 else None
+    init = _normal(rng, (N,)) if with_init else None
+    return {"a": a, "b": b, "reset": reset, "init": init}

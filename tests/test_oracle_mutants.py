@@ -42,6 +42,9 @@ MUTANTS = {
                                 "if (te[t] || (tr && tr[t])) prev = 0.0;"),
     "prefix_ignores_truncation": ("if (t > 0 && (te[t - 1] || (tr && tr[t - 1]))) s = 0;",
                                   "if (t > 0 && te[t - 1]) s = 0;"),
+    "affine_reset_ignored": ("if (!(reset && reset[i])) v += (double)a[i] * carry;",
+                             "v += (double)a[i] * carry;"),
+    "affine_init_ignored": ("double carry = init ? (double)init[n] : 0.0;", "double carry = 0.0;"),
 }
 
 PIN_TESTS = [
@@ -53,6 +56,8 @@ PIN_TESTS = [
     lambda: pins.test_retrace_matches_munos_sum(3),
     lambda: pins.test_elig_matches_episode_sum(True),
     lambda: pins.test_prefix_sum_matches_episode_sum(),
+    lambda: pins.test_affine_matches_bruteforce_sum(True, True),
+    lambda: pins.test_affine_every_reset_pattern(False),
 ]
 
 

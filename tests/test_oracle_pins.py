@@ -504,3 +504,108 @@ def test_prefix_sum_stays_in_int32_at_workload_sizes():
     d = synthetic.workload_inputs("long_256x16384", "episodic_prefix_sum")
     _, mx = oracle.episodic_prefix_sum(d["x"], d["terminated"], d["truncated"])
     assert mx < 2 ** 31 - 1
+
+
+# --------------------------------------------------------------------------
+# the generic affine scan x_t = b_t + a_t x_prev (unified recurrence,
+# gist.science technical summary, Methodologie 1, coefficients given)
+# --------------------------------------------------------------------------
+
+def bf_affine(a, b, reset, init, reverse):
+    """Non-recursive: x at scan position p is the sum, over the positions q of
+    p's segment (back to the nearest reset, or the row start), of b_q times
+    the product of a over (q, p]; when the segment reaches the row start
+    without a reset, init times the product of a over [0, p] is added."""
+    N, T = a.shape
+    out = np.zeros((N, T))
+    for n in range(N):
+        idx = list(range(T - 1, -1, -1)) if reverse else list(range(T))
+        rs = [bool(reset is not None and reset[n, t]) for t in idx]
+        for pos in range(T):
+            start = pos
+            while start > 0 and not rs[start]:
+                start -= 1
+            total = 0.0
+            for q in range(start, pos + 1):
+                total += float(b[n, idx[q]]) * float(np.prod([float(a[n, idx[u]]) for u in range(q + 1, pos + 1)]))
+            if not rs[start] and init is not None:
+                total += float(init[n]) * float(np.prod([float(a[n, idx[u]]) for u in range(0, pos + 1)]))
+            out[n, idx[pos]] = total
+    return out
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("with_init", [False, True])
+def test_affine_matches_bruteforce_sum(reverse, with_init):
+    d = synthetic.make_affine_inputs(4, 9, seed=31, p_reset=0.2, with_init=with_init, a_low=-1.2, a_high=1.2)
+    got = oracle.affine_scan(d["a"], d["b"], d["reset"], d["init"], reverse=reverse)
+    np.testing.assert_allclose(got, bf_affine(d["a"], d["b"], d["reset"], d["init"], reverse),
+                               rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_affine_every_reset_pattern(reverse):
+    T = 5
+    rng = np.random.default_rng(5)
+    a = rng.uniform(-1, 1, (1, T)).astype(np.float32)
+    b = rng.standard_normal((1, T)).astype(np.float32)
+    init = rng.standard_normal(1).astype(np.float32)
+    for bits in itertools.product([0, 1], repeat=T):
+        reset = np.array([bits], np.uint8)
+        got = oracle.affine_scan(a, b, reset, init, reverse=reverse)
+        np.testing.assert_allclose(got, bf_affine(a, b, reset, init, reverse), rtol=1e-12, atol=1e-12)
+
+
+def test_affine_unit_coefficient_is_cumulative_sum():
+    d = synthetic.make_affine_inputs(3, 50, seed=32, p_reset=0.0, with_init=False)
+    ones = np.ones_like(d["a"])
+    np.testing.assert_allclose(oracle.affine_scan(ones, d["b"]), np.cumsum(d["b"].astype(np.float64), axis=1),
+                               rtol=1e-12, atol=1e-12)
+    rev = np.cumsum(d["b"][:, ::-1].astype(np.float64), axis=1)[:, ::-1]
+    np.testing.assert_allclose(oracle.affine_scan(ones, d["b"], reverse=True), rev, rtol=1e-12, atol=1e-12)
+
+
+def test_affine_zero_coefficient_returns_b():
+    d = synthetic.make_affine_inputs(2, 17, seed=33, p_reset=0.1)
+    for rev in (False, True):
+        got = oracle.affine_scan(np.zeros_like(d["a"]), d["b"], d["reset"], d["init"], reverse=rev)
+        np.testing.assert_array_equal(got, d["b"].astype(np.float64))
+
+
+@pytest.mark.parametrize("c", [0.5, 0.99, -0.7])
+def test_affine_constant_coefficient_geometric_sum(c):
+    T = 40
+    a = np.full((1, T), c, np.float32)
+    b = np.ones((1, T), np.float32)
+    cc = float(np.float32(c))
+    k = np.arange(T, dtype=np.float64)
+    want = (1.0 - cc ** (k + 1)) / (1.0 - cc)
+    np.testing.assert_allclose(oracle.affine_scan(a, b)[0], want, rtol=1e-12)
+    np.testing.assert_allclose(oracle.affine_scan(a, b, reverse=True)[0], want[::-1], rtol=1e-12)
+
+
+def test_affine_backward_is_forward_on_reversed_rows():
+    d = synthetic.make_affine_inputs(5, 64, seed=34, p_reset=0.05)
+    fl = lambda x: None if x is None else np.ascontiguousarray(x[:, ::-1])  # noqa: E731
+    back = oracle.affine_scan(d["a"], d["b"], d["reset"], d["init"], reverse=True)
+    fwd = oracle.affine_scan(fl(d["a"]), fl(d["b"]), fl(d["reset"]), d["init"])
+    np.testing.assert_array_equal(back, fwd[:, ::-1])
+
+
+def test_affine_reproduces_discounted_return():
+    # discounted return = backward scan with a = gamma cont, b = r + gamma (1 - cont) nv
+    d = synthetic.make_inputs("discounted_return", 6, 30, seed=35, p_term=0.1)
+    r, term, boot = d["rewards"], d["terminated"], d["bootstrap"]
+    g = float(np.float32(0.97))
+    want = oracle.discounted_return(r, boot, term, None, None, gamma=g)
+    cont = (term == 0).astype(np.float64)
+    cont[:, -1] = 0.0
+    nv = np.where(term != 0, 0.0, np.broadcast_to(boot.astype(np.float64)[:, None], r.shape))
+    a = (g * cont).astype(np.float64)
+    b = r.astype(np.float64) + g * (1.0 - cont) * nv
+    got = bf_affine(a, b, None, None, reverse=True)
+    np.testing.assert_allclose(want, got, rtol=1e-9, atol=1e-9)
+    # and the oracle's own scan on the same (fp32-representable) coefficients
+    a32, b32 = a.astype(np.float32), b.astype(np.float32)
+    np.testing.assert_allclose(oracle.affine_scan(a32, b32, reverse=True), bf_affine(a32, b32, None, None, True),
+                               rtol=1e-12, atol=1e-12)

@@ -49,6 +49,10 @@ def algorithmic_bytes(est: str, d: dict) -> int:
     `trunc_value` is counted only where truncated (one 32-byte sector each);
     per-row arrays (bootstrap, init_trace) count 4 B per row; every output
     counts 4 B per step."""
+    if est == "affine_scan":  # a, b, reset flags, init per row, one output
+        N, T = d["a"].shape
+        return int(8 * N * T + (N * T if d.get("reset") is not None else 0)
+                   + (4 * N if d.get("init") is not None else 0) + 4 * N * T)
     if est == "retrace":
         N, T, A = d["q"].shape
     else:
@@ -188,10 +192,11 @@ ARG_ORDER = {
     "discounted_return": ("rewards", "bootstrap", "terminated", "truncated", "trunc_value"),
     "elig_trace": ("inputs", "init_trace", "terminated", "truncated"),
     "episodic_prefix_sum": ("x", "terminated", "truncated"),
+    "affine_scan": ("a", "b", "reset", "init"),
 }
 OUT_KW = {"gae": ("advantages", "returns"), "vtrace": ("vs", "pg_advantages"), "retrace": ("q_ret",),
           "td_lambda": ("returns",), "discounted_return": ("returns",), "elig_trace": ("traces",),
-          "episodic_prefix_sum": ("out",)}
+          "episodic_prefix_sum": ("out",), "affine_scan": ("x",)}
 
 
 def workload_calls(workload: str, rank: int):
@@ -201,8 +206,11 @@ def workload_calls(workload: str, rank: int):
     for est in w["estimators"]:
         for T in w["Ts"]:
             seed = shard_seed(synthetic.seed_for(workload, est, T), rank)
-            d = synthetic.make_inputs(est, w["N"], T, seed=seed, p_term=w["p_term"],
-                                      p_trunc=w["p_trunc"], A=w.get("A", 18))
+            if est == "affine_scan":
+                d = synthetic.make_affine_inputs(w["N"], T, seed=seed, p_reset=w["p_term"])
+            else:
+                d = synthetic.make_inputs(est, w["N"], T, seed=seed, p_term=w["p_term"],
+                                          p_trunc=w["p_trunc"], A=w.get("A", 18))
             calls.append((est, T, d))
     return calls
 

@@ -216,6 +216,23 @@ rlscan_status rlscan_episodic_prefix_sum(const int32_t *x, const uint8_t *termin
                                          int64_t T, rlscan_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Generic affine scan: the recurrence every estimator above specialises
+ * (gist.science technical summary, Methodologie 1: A_t = alpha_t +
+ * beta_t A_{t+1} and its forward-time mirror), with the coefficients given
+ * instead of built.  In scan order -- t = 0..T-1, or t = T-1..0 when
+ * `reverse` is 1 --
+ *   x_t = b_t + a_t * x_prev,
+ * where x_prev is the previous step in scan order, or init[n] for the row's
+ * first step (init nullable: 0).  reset[t] != 0 cuts the dependency:
+ * x_t = b_t (reset nullable: no resets).  Rows are independent.
+ * Inputs  a, b [N,T] float32; reset [N,T] uint8 (nullable); init [N] (nullable).
+ * Output  x [N,T] float32.
+ * Errors  RLSCAN_ERR_INVALID_ARG also for reverse other than 0 or 1.
+ * ------------------------------------------------------------------------- */
+rlscan_status rlscan_affine_scan(const float *a, const float *b, const uint8_t *reset, const float *init,
+                                 float *x, int64_t N, int64_t T, int32_t reverse, rlscan_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Status, workspace and configuration.
  * ------------------------------------------------------------------------- */
 
@@ -248,7 +265,8 @@ typedef enum rlscan_estimator {
   RLSCAN_EST_TD_LAMBDA = 3,
   RLSCAN_EST_DISCOUNTED_RETURN = 4,
   RLSCAN_EST_ELIG_TRACE = 5,
-  RLSCAN_EST_EPISODIC_PREFIX_SUM = 6
+  RLSCAN_EST_EPISODIC_PREFIX_SUM = 6,
+  RLSCAN_EST_AFFINE_SCAN = 7
 } rlscan_estimator;
 
 /* How a call of the given shape is executed (no device work, no allocation). */

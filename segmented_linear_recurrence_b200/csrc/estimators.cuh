@@ -467,4 +467,56 @@ struct PrefixSumOp {
   }
 };
 
+// ---------------------------------------------------------------------------
+// Generic affine scan: the pages' unified recurrence with its coefficients
+// given (gist.science technical summary, Methodologie 1).  In scan order
+// (forward, or backward when BWD) x_t = b_t + a_t x_prev; reset[t] cuts the
+// dependency (a = 0, x = b); the row's first step in scan order -- its
+// dependency edge -- takes the per-row initial carry in its local term:
+// b + a init (init NULL: 0).  The reset flags travel in the flag slot of
+// `term`; `trunc` is NULL.
+// ---------------------------------------------------------------------------
+template <bool BWD>
+struct AffineOp {
+  static constexpr int kRegs = 40, kRegsLookback = 40;  // registers per thread, chosen by measurement
+  using V = float;
+  static constexpr bool kBackward = BWD;
+  struct Args {
+    const float *a, *b, *init;
+    const uint8_t *term, *trunc;  // term: reset flags (nullable); trunc: NULL
+    float *out;
+  };
+  struct Raw {
+    float a[8], b[8];
+    Flags f;
+    float ev;  // init of the tile's row edge
+  };
+  static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int, uint32_t,
+                                              Flags f, Raw &w) {
+    ld8(p.a, tl, w.a);
+    ld8(p.b, tl, w.b);
+    w.f = f;
+    w.ev = edge_value(p.init, tl, fd);
+  }
+  static __device__ __forceinline__ void fetch_boundary(const Args &, const Tile &, const FastDiv &, Raw &) {}
+  static __device__ __forceinline__ float nbr_of(const Raw &) { return 0.0f; }
+  static __device__ __forceinline__ float halo_of(const Raw &) { return 0.0f; }
+  static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w, float,
+                                              Aff<float> (&c)[8]) {
+    const uint32_t cut = w.f.term | tl.edge;
+    const uint32_t init_at = tl.edge & ~w.f.term;  // edge steps that take the initial carry
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float b = w.b[k];
+      if (((init_at >> k) & 1u) && p.init)
+        b = fmaf(w.a[k], tl.few_rows ? w.ev : __ldg(p.init + tl.n0 + fd.div(tl.t0 + k)), b);
+      c[k] = Aff<float>{((cut >> k) & 1u) ? 0.0f : w.a[k], b};
+    }
+  }
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[8],
+                                              const float (&x)[8], const float (&)[8]) {
+    st8(p.out, tl, x);
+  }
+};
+
 }  // namespace rlscan

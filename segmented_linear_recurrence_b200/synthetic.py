@@ -33,6 +33,7 @@ SCALARS = {
     "retrace": dict(gamma=0.99, lam=0.95),
     "elig_trace": dict(gamma=0.99, lam=0.95),
     "episodic_prefix_sum": dict(),
+    "affine_scan": dict(reverse=True),
 }
 
 SWEEP_T = (32, 64, 128, 256, 512, 1024, 2048)
@@ -49,12 +50,16 @@ WORKLOADS = {
                                 p_trunc=0.0, A=18),
     "long_256x16384": dict(index=4, N=256, Ts=(16384,), estimators=ESTIMATORS, p_term=0.01,
                            p_trunc=0.0, A=6),
+    # the generic affine scan (backward), resets at p_term
+    "affine_4096xT": dict(index=5, N=4096, Ts=(512, 2048), estimators=("affine_scan",), p_term=0.01,
+                          p_trunc=0.0),
 }
 
 
 def seed_for(workload: str, estimator: str, T: int) -> int:
     w = WORKLOADS[workload]
-    return 1000 + 100 * w["index"] + 10 * list(w["Ts"]).index(T) + ESTIMATORS.index(estimator)
+    k = ESTIMATORS.index(estimator) if estimator in ESTIMATORS else len(ESTIMATORS)
+    return 1000 + 100 * w["index"] + 10 * list(w["Ts"]).index(T) + k
 
 
 def _normal(rng, shape):
@@ -115,6 +120,8 @@ def workload_inputs(workload: str, estimator: str, T: int | None = None) -> dict
     """Inputs of one estimator in a named workload (first T if not given)."""
     w = WORKLOADS[workload]
     T = w["Ts"][0] if T is None else T
+    if estimator == "affine_scan":
+        return make_affine_inputs(w["N"], T, seed=seed_for(workload, estimator, T), p_reset=w["p_term"])
     return make_inputs(estimator, w["N"], T, seed=seed_for(workload, estimator, T),
                        p_term=w["p_term"], p_trunc=w["p_trunc"], A=w.get("A", 18))
 

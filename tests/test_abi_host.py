@@ -183,3 +183,18 @@ def test_binding_raises_without_gpu():
     r = torch.zeros(2, 4)
     with pytest.raises(RuntimeError):
         slr.rlscan_discounted_return(r, None, torch.zeros(2, 4, dtype=torch.uint8))
+
+
+def test_affine_scan_argument_checks(L):
+    a, b, x = P(BASE), P(BASE + 0x10000), P(BASE + 0x20000)
+    assert L.rlscan_affine_scan(None, None, None, None, None, 0, 5, 0, None) == OK  # empty
+    assert L.rlscan_affine_scan(a, b, None, None, x, 4, 8, 2, None) == INVALID  # direction
+    assert L.rlscan_affine_scan(a, b, None, None, x, 4, 8, -1, None) == INVALID
+    assert L.rlscan_affine_scan(None, b, None, None, x, 4, 8, 0, None) == INVALID  # a required
+    assert L.rlscan_affine_scan(a, None, None, None, x, 4, 8, 0, None) == INVALID  # b required
+    assert L.rlscan_affine_scan(a, b, None, None, None, 4, 8, 1, None) == INVALID  # x required
+    assert L.rlscan_affine_scan(a, b, None, None, P(BASE + 2), 4, 8, 1, None) == INVALID  # misaligned
+    assert L.rlscan_affine_scan(a, b, None, None, a, 4, 8, 1, None) == OVERLAP  # in place
+    p = slr.rlscan_query_plan("affine_scan", 4096, 2000)
+    assert p["lookback"] == 0 and p["chunk_steps"] % 2000 == 0
+    assert slr.rlscan_query_plan("affine_scan", 2, 100000)["lookback"] == 1

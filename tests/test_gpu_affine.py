@@ -1,0 +1,131 @@
+"""GPU parity of the generic affine scan (rlscan_affine_scan) against the
+oracle: x_t = b_t + a_t x_prev along T, forward or backward, with resets and
+a per-row initial carry.  Same bar as the estimators: |gpu - ref| <= 1e-4 (1 +
+|ref|) element by element, on every plan (whole-row blocks of every size,
+look-back chains), odd and long rows, unaligned views and host tensors."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import segmented_linear_recurrence_b200 as slr
+from segmented_linear_recurrence_b200 import build as slr_build
+from segmented_linear_recurrence_b200 import synthetic
+
+from .util import TOL
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    slr_build.build()
+
+
+@pytest.fixture
+def options():
+    yield slr.rlscan_set_option
+    for name, default in (("force_lookback", 0), ("force_block", 0), ("force_scalar", 0)):
+        slr.rlscan_set_option(name, default)
+
+
+def run_both(d, reverse, device="cuda", views=None):
+    t = {k: None if v is None else torch.from_numpy(np.ascontiguousarray(v)).to(device) for k, v in d.items()}
+    if views is not None:
+        t = views(t)
+    got = slr.rlscan_affine_scan(t["a"], t["b"], t["reset"], t["init"], reverse=reverse)
+    ref = oracle.affine_scan(d["a"], d["b"], d["reset"], d["init"], reverse=reverse)
+    return got.cpu().numpy().astype(np.float64), ref
+
+
+def assert_close(got, ref, what):
+    err = np.abs(got - ref)
+    bound = TOL * (1.0 + np.abs(ref))
+    bad = np.argwhere(err > bound)
+    assert bad.size == 0, f"{what}: {bad.shape[0]} elements off, first {tuple(bad[0])}: " \
+                          f"gpu {got[tuple(bad[0])]} ref {ref[tuple(bad[0])]}"
+
+
+CASES = [(512, 128), (64, 2048), (4096, 512), (5, 5000), (40, 96), (33, 1001), (7, 3), (1, 70001), (3, 1)]
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("N,T", CASES)
+def test_affine_matches_oracle(N, T, reverse):
+    d = synthetic.make_affine_inputs(N, T, seed=2000 + N + T, p_reset=0.01)
+    got, ref = run_both(d, reverse)
+    assert_close(got, ref, f"N={N} T={T} reverse={reverse}")
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("with_reset,with_init", [(False, False), (False, True), (True, False)])
+def test_affine_optional_inputs(reverse, with_reset, with_init):
+    d = synthetic.make_affine_inputs(96, 777, seed=2101, p_reset=0.02 if with_reset else 0.0,
+                                     with_init=with_init)
+    got, ref = run_both(d, reverse)
+    assert_close(got, ref, f"reset={with_reset} init={with_init}")
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("block", [128, 192, 256, 384, 512])
+@pytest.mark.parametrize("lookback", [0, 1])
+def test_affine_every_plan(reverse, block, lookback, options):
+    options("force_block", block)
+    options("force_lookback", lookback)
+    for N, T in ((100, 100), (3, 9000), (17, 1537)):
+        d = synthetic.make_affine_inputs(N, T, seed=2200 + N, p_reset=0.01)
+        got, ref = run_both(d, reverse)
+        assert_close(got, ref, f"block={block} lookback={lookback} N={N} T={T}")
+
+
+def test_affine_unit_coefficient_long_row_is_cumsum():
+    # a = 1 without resets: the cumulative sum of b over a row of 2^20 steps,
+    # a chain of 512 look-back chunks.  b >= 0 so the sums do not cancel: with
+    # a = 1 the fp32 error grows with the partial sums, and a zero-mean sum
+    # near a crossing of 0 is ill-conditioned for any fp32 evaluation order.
+    d = synthetic.make_affine_inputs(2, 1 << 20, seed=2301, p_reset=0.0, with_init=False)
+    d["a"][:] = 1.0
+    d["b"] = np.abs(d["b"])
+    for reverse in (False, True):
+        got, ref = run_both(d, reverse)
+        assert_close(got, ref, f"cumsum reverse={reverse}")
+
+
+def test_affine_unaligned_views_and_scalar_path(options):
+    d = synthetic.make_affine_inputs(20, 301, seed=2401, p_reset=0.03)
+
+    def shift(t):
+        # views starting one element in: no 32-byte alignment anywhere
+        out = {}
+        for k, v in t.items():
+            if v is None:
+                out[k] = None
+                continue
+            big = torch.empty(v.numel() + 1, dtype=v.dtype, device=v.device)
+            big[1:] = v.reshape(-1)
+            out[k] = big[1:].view(v.shape)
+        return out
+
+    for reverse in (False, True):
+        got, ref = run_both(d, reverse, views=shift)
+        assert_close(got, ref, f"unaligned reverse={reverse}")
+    options("force_scalar", 1)
+    got, ref = run_both(d, True)
+    assert_close(got, ref, "scalar path")
+
+
+def test_affine_host_tensors():
+    d = synthetic.make_affine_inputs(8, 500, seed=2501, p_reset=0.02)
+    got, ref = run_both(d, True, device="cpu")
+    assert_close(got, ref, "host tensors")
+
+
+def test_affine_reset_everywhere_returns_b():
+    d = synthetic.make_affine_inputs(16, 1000, seed=2601, p_reset=0.0)
+    d["reset"] = np.ones_like(d["a"], dtype=np.uint8)
+    for reverse in (False, True):
+        got, _ = run_both(d, reverse)
+        np.testing.assert_array_equal(got, d["b"].astype(np.float64))
+

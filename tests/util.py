@@ -15,6 +15,7 @@ OUTPUT_NAMES = {
     "discounted_return": ("returns",),
     "elig_trace": ("traces",),
     "episodic_prefix_sum": ("out",),
+    "affine_scan": ("x",),
 }
 
 
@@ -59,6 +60,9 @@ def gpu_run(est, d, stream=None, **scal):
     elif est == "episodic_prefix_sum":
         res = slr.rlscan_episodic_prefix_sum(t["x"], t["terminated"], t.get("truncated"),
                                              stream=stream)
+    elif est == "affine_scan":
+        res = slr.rlscan_affine_scan(t["a"], t["b"], t.get("reset"), t.get("init"),
+                                     reverse=bool(scal.get("reverse", False)), stream=stream)
     else:
         raise ValueError(est)
     res = res if isinstance(res, tuple) else (res,)

@@ -34,6 +34,7 @@ def bind(lib):
         "rlo_elig_trace": [i64, i64, vp, vp, vp, vp, dbl, dbl, vp],
         "rlo_episodic_prefix_sum": [i64, i64, vp, vp, vp, vp, vp],
         "rlo_affine_scan": [i64, i64, vp, vp, vp, vp, ctypes.c_int, vp],
+        "rlo_affine_scan_grad": [i64, i64, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -173,6 +174,22 @@ def affine_scan(a, b, reset=None, init=None, reverse=False):
     return out
 
 
+def affine_scan_grad(a, x, dy, reset=None, init=None, reverse=False):
+    """Adjoint of affine_scan: returns (da, db, dinit) for upstream dy, given
+    the forward output x (all fp64)."""
+    N, T = _dims(a)
+    keep = [_p(a, np.float32), _p(x, np.float32), _p(dy, np.float32), _p(reset, np.uint8),
+            _p(init, np.float32)]
+    da = np.empty((N, T), np.float64)
+    db = np.empty((N, T), np.float64)
+    dinit = np.empty((N,), np.float64)
+    rc = _load().rlo_affine_scan_grad(N, T, *[k[1] for k in keep], 1 if reverse else 0,
+                                      da.ctypes.data_as(ctypes.c_void_p), db.ctypes.data_as(ctypes.c_void_p),
+                                      dinit.ctypes.data_as(ctypes.c_void_p))
+    _check(rc, "affine_scan_grad")
+    return da, db, dinit
+
+
 # Convenience: dispatch by estimator name on a dict of inputs as produced by
 # segmented_linear_recurrence_b200.synthetic (keys match parameter names).
 def run(name, inp, **scal):
@@ -186,4 +203,4 @@ def run(name, inp, **scal):
 
 
 __all__ = ["gae", "td_lambda", "discounted_return", "vtrace", "retrace", "elig_trace",
-           "episodic_prefix_sum", "affine_scan", "run"]
+           "episodic_prefix_sum", "affine_scan", "affine_scan_grad", "run"]

@@ -316,3 +316,45 @@ int rlo_affine_scan(int64_t N, int64_t T, const float *a, const float *b,
   }
   return 0;
 }
+
+/* Gradient (adjoint) of rlo_affine_scan for a loss whose direct derivative
+ * with respect to x_t is dy_t.  x is the forward scan's output.  In the
+ * forward scan's order, with nxt(t) the following step and prv(t) the
+ * preceding one:
+ *   g_t   = dy_t + [nxt(t) exists and not reset] a_nxt(t) g_nxt(t)
+ *   db_t  = g_t
+ *   da_t  = [not reset_t] g_t * (x_prv(t), or init[n] at the first step)
+ *   dinit = [not reset at the first step] a_first g_first
+ * (the chain rule through the recurrence, evaluated last step first).
+ * da and dinit may be NULL. */
+int rlo_affine_scan_grad(int64_t N, int64_t T, const float *a, const float *x,
+                         const float *dy, const uint8_t *reset, const float *init,
+                         int reverse, double *da, double *db, double *dinit) {
+  if (bad_dims(N, T)) return -1;
+  for (int64_t n = 0; n < N; ++n) {
+    double g_next = 0.0, a_next = 0.0;
+    int have_next = 0, reset_next = 0;
+    for (int64_t k = T - 1; k >= 0; --k) { /* scan position k, last first */
+      const int64_t t = reverse ? T - 1 - k : k;
+      const int64_t i = n * T + t;
+      double g = (double)dy[i];
+      if (have_next && !reset_next) g += a_next * g_next;
+      db[i] = g;
+      const int r = reset && reset[i];
+      if (da) {
+        double xp;
+        if (k == 0)
+          xp = init ? (double)init[n] : 0.0;
+        else
+          xp = (double)x[n * T + (reverse ? t + 1 : t - 1)];
+        da[i] = r ? 0.0 : g * xp;
+      }
+      if (k == 0 && dinit) dinit[n] = r ? 0.0 : (double)a[i] * g;
+      g_next = g;
+      a_next = (double)a[i];
+      reset_next = r;
+      have_next = 1;
+    }
+  }
+  return 0;
+}

@@ -45,6 +45,10 @@ MUTANTS = {
     "affine_reset_ignored": ("if (!(reset && reset[i])) v += (double)a[i] * carry;",
                              "v += (double)a[i] * carry;"),
     "affine_init_ignored": ("double carry = init ? (double)init[n] : 0.0;", "double carry = 0.0;"),
+    "affine_grad_reset_ignored": ("if (have_next && !reset_next) g += a_next * g_next;",
+                                  "if (have_next) g += a_next * g_next;"),
+    "affine_grad_wrong_neighbour": ("xp = (double)x[n * T + (reverse ? t + 1 : t - 1)];",
+                                    "xp = (double)x[n * T + (reverse ? t - 1 : t + 1)];"),
 }
 
 PIN_TESTS = [
@@ -58,6 +62,8 @@ PIN_TESTS = [
     lambda: pins.test_prefix_sum_matches_episode_sum(),
     lambda: pins.test_affine_matches_bruteforce_sum(True, True),
     lambda: pins.test_affine_every_reset_pattern(False),
+    lambda: pins.test_affine_grad_matches_finite_differences(False, 0.3),
+    lambda: pins.test_affine_grad_matches_finite_differences(True, 0.3),
 ]
 
 

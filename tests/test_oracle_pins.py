@@ -609,3 +609,68 @@ def test_affine_reproduces_discounted_return():
     a32, b32 = a.astype(np.float32), b.astype(np.float32)
     np.testing.assert_allclose(oracle.affine_scan(a32, b32, reverse=True), bf_affine(a32, b32, None, None, True),
                                rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# adjoint of the affine scan: pinned against central finite differences of
+# the non-recursive forward sum (bf_affine), never against its own recursion
+# --------------------------------------------------------------------------
+
+def _fd_grads(a, b, reset, init, w, reverse, h=1e-5):
+    """Gradients of L = sum(w * x) by central differences of bf_affine in fp64."""
+    a64, b64 = a.astype(np.float64), b.astype(np.float64)
+    i64 = None if init is None else init.astype(np.float64)
+    L = lambda aa, bb, ii: float(np.sum(w * bf_affine(aa, bb, reset, ii, reverse)))  # noqa: E731
+    da, db = np.zeros_like(a64), np.zeros_like(b64)
+    for idx in np.ndindex(*a.shape):
+        for arr, out in ((a64, da), (b64, db)):
+            p, m = arr.copy(), arr.copy()
+            p[idx] += h
+            m[idx] -= h
+            args_p = (p, b64, i64) if arr is a64 else (a64, p, i64)
+            args_m = (m, b64, i64) if arr is a64 else (a64, m, i64)
+            out[idx] = (L(*args_p) - L(*args_m)) / (2 * h)
+    dinit = np.zeros(a.shape[0])
+    if i64 is not None:
+        for n in range(a.shape[0]):
+            p, m = i64.copy(), i64.copy()
+            p[n] += h
+            m[n] -= h
+            dinit[n] = (L(a64, b64, p) - L(a64, b64, m)) / (2 * h)
+    return da, db, dinit
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("p_reset", [0.0, 0.3])
+def test_affine_grad_matches_finite_differences(reverse, p_reset):
+    d = synthetic.make_affine_inputs(3, 7, seed=41, p_reset=p_reset, a_low=-1.1, a_high=1.1)
+    w = np.random.default_rng(42).standard_normal((3, 7)).astype(np.float32)
+    x = oracle.affine_scan(d["a"], d["b"], d["reset"], d["init"], reverse=reverse).astype(np.float32)
+    da, db, dinit = oracle.affine_scan_grad(d["a"], x, w, d["reset"], d["init"], reverse=reverse)
+    fda, fdb, fdinit = _fd_grads(d["a"], d["b"], d["reset"], d["init"], w.astype(np.float64), reverse)
+    np.testing.assert_allclose(db, fdb, rtol=1e-6, atol=1e-6)
+    np.testing.assert_allclose(da, fda, rtol=1e-5, atol=1e-5)  # x passed as fp32
+    np.testing.assert_allclose(dinit, fdinit, rtol=1e-6, atol=1e-6)
+
+
+def test_affine_grad_unit_coefficient_is_reverse_cumsum():
+    d = synthetic.make_affine_inputs(2, 40, seed=43, p_reset=0.0, with_init=False)
+    a = np.ones_like(d["a"])
+    dy = d["b"]
+    x = oracle.affine_scan(a, d["b"]).astype(np.float32)
+    _, db, _ = oracle.affine_scan_grad(a, x, dy)
+    np.testing.assert_allclose(db, np.cumsum(dy[:, ::-1].astype(np.float64), axis=1)[:, ::-1], rtol=1e-12)
+    _, db_r, _ = oracle.affine_scan_grad(a, x, dy, reverse=True)
+    np.testing.assert_allclose(db_r, np.cumsum(dy.astype(np.float64), axis=1), rtol=1e-12)
+
+
+def test_affine_grad_zero_coefficient():
+    d = synthetic.make_affine_inputs(2, 9, seed=44, p_reset=0.0)
+    a = np.zeros_like(d["a"])
+    x = oracle.affine_scan(a, d["b"], None, d["init"]).astype(np.float32)
+    dy = d["b"]
+    da, db, dinit = oracle.affine_scan_grad(a, x, dy, None, d["init"])
+    np.testing.assert_array_equal(db, dy.astype(np.float64))
+    xp = np.concatenate([d["init"][:, None], x[:, :-1]], axis=1).astype(np.float64)
+    np.testing.assert_allclose(da, dy.astype(np.float64) * xp, rtol=1e-15)
+    np.testing.assert_array_equal(dinit, np.zeros(2))

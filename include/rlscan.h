@@ -233,6 +233,23 @@ rlscan_status rlscan_affine_scan(const float *a, const float *b, const uint8_t *
                                  float *x, int64_t N, int64_t T, int32_t reverse, rlscan_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Gradient of rlscan_affine_scan (its adjoint), for a loss L whose direct
+ * derivative with respect to x_t is dy_t.  `x` is the forward call's output
+ * and `reverse` its direction.  The chain rule through the recurrence is an
+ * affine scan in the opposite direction: with nxt(t) / prv(t) the following
+ * / preceding step in the forward scan's order,
+ *   g_t      = dy_t + a_nxt(t) g_nxt(t)   (0 term if nxt(t) resets or is absent)
+ *   db_t     = g_t                                          dL/db
+ *   da_t     = g_t * x_prv(t), x_prv = init[n] at the first step, 0 where reset
+ *   dinit[n] = a_first g_first, 0 if the first step resets  dL/dinit
+ * Inputs  a, x, dy [N,T] float32; reset [N,T] (nullable); init [N] (nullable).
+ * Output  db [N,T]; da [N,T] (nullable); dinit [N] (nullable).
+ * ------------------------------------------------------------------------- */
+rlscan_status rlscan_affine_scan_grad(const float *a, const float *x, const float *dy, const uint8_t *reset,
+                                      const float *init, float *da, float *db, float *dinit, int64_t N,
+                                      int64_t T, int32_t reverse, rlscan_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Status, workspace and configuration.
  * ------------------------------------------------------------------------- */
 
@@ -266,7 +283,8 @@ typedef enum rlscan_estimator {
   RLSCAN_EST_DISCOUNTED_RETURN = 4,
   RLSCAN_EST_ELIG_TRACE = 5,
   RLSCAN_EST_EPISODIC_PREFIX_SUM = 6,
-  RLSCAN_EST_AFFINE_SCAN = 7
+  RLSCAN_EST_AFFINE_SCAN = 7,
+  RLSCAN_EST_AFFINE_SCAN_GRAD = 8
 } rlscan_estimator;
 
 /* How a call of the given shape is executed (no device work, no allocation). */

@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "RlscanError", "lib", "rlscan_gae", "rlscan_vtrace", "rlscan_retrace", "rlscan_td_lambda",
     "rlscan_discounted_return", "rlscan_elig_trace", "rlscan_episodic_prefix_sum",
-    "rlscan_affine_scan", "rlscan_sync_status", "rlscan_status_string", "rlscan_release_workspaces",
+    "rlscan_affine_scan", "rlscan_affine_scan_grad", "rlscan_sync_status", "rlscan_status_string", "rlscan_release_workspaces",
     "rlscan_abi_version", "rlscan_query_plan", "rlscan_set_option", "rlscan_get_option",
     "rlscan_reserve_workspace",
     "STATUS", "OPTIONS", "ESTIMATOR_IDS", "LIB_PATH",
@@ -36,7 +36,7 @@ STATUS = {0: "RLSCAN_OK", 1: "RLSCAN_ERR_INVALID_ARG", 2: "RLSCAN_ERR_OVERLAP",
 OPTIONS = {"lookback_timeout_ns": 1, "force_lookback": 2, "force_block": 3, "force_scalar": 4,
            "check_pointers": 5, "test_starve_lookback": 6, "pdl": 7}
 ESTIMATOR_IDS = {"gae": 0, "vtrace": 1, "retrace": 2, "td_lambda": 3, "discounted_return": 4,
-                 "elig_trace": 5, "episodic_prefix_sum": 6, "affine_scan": 7}
+                 "elig_trace": 5, "episodic_prefix_sum": 6, "affine_scan": 7, "affine_scan_grad": 8}
 
 
 class RlscanError(RuntimeError):
@@ -62,6 +62,7 @@ _SIGNATURES = {
     "rlscan_elig_trace": [_VP] * 5 + [_I64, _I64, _F, _F, _VP],
     "rlscan_episodic_prefix_sum": [_VP] * 4 + [_I64, _I64, _VP],
     "rlscan_affine_scan": [_VP] * 5 + [_I64, _I64, ctypes.c_int32, _VP],
+    "rlscan_affine_scan_grad": [_VP] * 8 + [_I64, _I64, ctypes.c_int32, _VP],
     "rlscan_sync_status": [_VP],
     "rlscan_release_workspaces": [],
     "rlscan_reserve_workspace": [_I64, _VP],
@@ -320,6 +321,26 @@ def rlscan_affine_scan(a, b, reset=None, init=None, *, reverse=False, x=None, st
     st = lib().rlscan_affine_scan(c.ptr(aa), c.ptr(bb), c.ptr(rs), c.ptr(x0), c.ptr(out), N, T,
                                   1 if reverse else 0, c.stream(stream))
     return c.finish(st, (out,))[0]
+
+
+def rlscan_affine_scan_grad(a, x, dy, reset=None, init=None, *, reverse=False, need_da=True,
+                            need_dinit=True, da=None, db=None, dinit=None, stream=None):
+    """Gradient of rlscan_affine_scan given the forward output `x` and the
+    upstream gradient `dy`.  Returns (da, db, dinit); da / dinit are None
+    when not requested."""
+    N, T = _nt(a, "rlscan_affine_scan_grad")
+    c = _Call("rlscan_affine_scan_grad", a)
+    aa = c.tensor(a, torch.float32, (N, T), "a")
+    xx = c.tensor(x, torch.float32, (N, T), "x")
+    gy = c.tensor(dy, torch.float32, (N, T), "dy")
+    rs = c.tensor(reset, torch.uint8, (N, T), "reset", required=False)
+    x0 = c.tensor(init, torch.float32, (N,), "init", required=False)
+    o_db = c.output(db, torch.float32, (N, T), "db")
+    o_da = c.output(da, torch.float32, (N, T), "da") if (need_da or da is not None) else None
+    o_di = c.output(dinit, torch.float32, (N,), "dinit") if (need_dinit or dinit is not None) else None
+    st = lib().rlscan_affine_scan_grad(c.ptr(aa), c.ptr(xx), c.ptr(gy), c.ptr(rs), c.ptr(x0), c.ptr(o_da),
+                                       c.ptr(o_db), c.ptr(o_di), N, T, 1 if reverse else 0, c.stream(stream))
+    return c.finish(st, (o_da, o_db, o_di))
 
 
 # ---------------------------------------------------------------------------

@@ -519,4 +519,115 @@ struct AffineOp {
   }
 };
 
+// ---------------------------------------------------------------------------
+// Adjoint of the generic affine scan (its gradient), for upstream gradients
+// dy and the forward output x of a scan in direction R (R: backward in t).
+// The chain rule through the recurrence is itself an affine scan, run in the
+// opposite direction:  g_t = dy_t + a'_t g_nxt,  a'_t = a_nxt unless the
+// following step in the forward order (nxt) resets or does not exist; then
+// db = g, da_t = g_t x_prv (0 where reset; x_prv = init[n] at the forward
+// scan's first step), dinit[n] = a g at that first step (0 if it resets).
+// ---------------------------------------------------------------------------
+template <bool R>
+struct AffineGradOp {
+  static constexpr int kRegs = 56, kRegsLookback = 56;  // registers per thread: no spills
+  using V = float;
+  static constexpr bool kBackward = !R;  // the adjoint runs against the forward scan
+  struct Args {
+    const float *a, *x, *dy, *init;
+    const uint8_t *term, *trunc;  // term: reset flags (nullable); trunc: NULL
+    float *da, *db, *dinit;       // da, dinit nullable
+    uint32_t T;
+  };
+  struct Raw {
+    float a[8], x[8], dy[8];
+    Flags f;
+    float ahalo;  // effective a (0 where reset) of the dependency neighbour past the tile
+    float xhalo;  // x of the neighbour past the tile on the other side
+    float iv;     // init of the row whose forward first step is in the tile (T >= 8)
+    uint32_t lane;
+  };
+  // Steps of the tile that are the forward scan's first step of their row.
+  static __device__ __forceinline__ uint32_t first_steps(const Tile &tl, uint32_t T) {
+    uint32_t e = 0;
+    if (tl.few_rows) {
+      if (R) {
+        const uint32_t rend = T - 1u - tl.t0;
+        e = rend < 8u ? (1u << rend) : 0u;
+      } else {
+        const uint32_t s = tl.t0 == 0u ? 0u : T - tl.t0;
+        e = s < 8u ? (1u << s) : 0u;
+      }
+    } else {
+      uint32_t tt = tl.t0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (R ? (tt == T - 1u) : (tt == 0u)) e |= 1u << k;
+        if (++tt == T) tt = 0;
+      }
+    }
+    return e & tl.valid;
+  }
+  static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int lane,
+                                              uint32_t total, Flags f, Raw &w) {
+    ld8(p.a, tl, w.a);
+    ld8(p.x, tl, w.x);
+    ld8(p.dy, tl, w.dy);
+    w.f = f;
+    w.lane = uint32_t(lane);
+    // dependency neighbour past the tile: t+1 (adjoint backward) / t-1 (forward)
+    w.ahalo = 0.0f;
+    if (!R && lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total)
+      w.ahalo = (p.term && __ldg(p.term + tl.i0 + 8u)) ? 0.0f : __ldg(p.a + tl.i0 + 8u);
+    if (R && lane == 0 && tl.i0 > 0u && tl.nvalid > 0)
+      w.ahalo = (p.term && __ldg(p.term + tl.i0 - 1u)) ? 0.0f : __ldg(p.a + tl.i0 - 1u);
+    // the other neighbour, for x_prv: t-1 (R false) / t+1 (R true)
+    w.xhalo = 0.0f;
+    if (!R && lane == 0 && tl.i0 > 0u && tl.nvalid > 0) w.xhalo = __ldg(p.x + tl.i0 - 1u);
+    if (R && lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total) w.xhalo = __ldg(p.x + tl.i0 + 8u);
+    w.iv = 0.0f;
+    const uint32_t fs = first_steps(tl, p.T);
+    if (p.init && tl.few_rows && fs) w.iv = __ldg(p.init + tl.n0 + fd.div(tl.t0 + uint32_t(__ffs(fs) - 1)));
+  }
+  static __device__ __forceinline__ void fetch_boundary(const Args &, const Tile &, const FastDiv &, Raw &) {}
+  // a' of the tile's first step in dependency order comes from the neighbour
+  static __device__ __forceinline__ float nbr_of(const Raw &w) {
+    return R ? (((w.f.term >> 7) & 1u) ? 0.0f : w.a[7]) : ((w.f.term & 1u) ? 0.0f : w.a[0]);
+  }
+  static __device__ __forceinline__ float halo_of(const Raw &w) { return w.ahalo; }
+  static __device__ __forceinline__ void coef(const Args &, const Tile &tl, const FastDiv &, Raw &w, float nb,
+                                              Aff<float> (&c)[8]) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float an;  // effective a of the following step in forward order
+      if (R)
+        an = k > 0 ? (((w.f.term >> (k - 1)) & 1u) ? 0.0f : w.a[k > 0 ? k - 1 : 0]) : nb;
+      else
+        an = k < 7 ? (((w.f.term >> (k + 1)) & 1u) ? 0.0f : w.a[k < 7 ? k + 1 : 7]) : nb;
+      c[k] = Aff<float>{((tl.edge >> k) & 1u) ? 0.0f : an, w.dy[k]};
+    }
+  }
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &w, const Aff<float> (&)[8],
+                                              const float (&g)[8], const float (&)[8]) {
+    st8(p.db, tl, g);
+    if (!p.da && !p.dinit) return;
+    // x_prv of each step: the other neighbour, by shuffle across the lane edge
+    const float mine = R ? w.x[0] : w.x[7];
+    float other = R ? __shfl_down_sync(0xffffffffu, mine, 1) : __shfl_up_sync(0xffffffffu, mine, 1);
+    if (R ? w.lane == 31u : w.lane == 0u) other = w.xhalo;
+    const uint32_t fs = first_steps(tl, p.T);
+    float da[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float xp = R ? (k < 7 ? w.x[k < 7 ? k + 1 : 7] : other) : (k > 0 ? w.x[k > 0 ? k - 1 : 0] : other);
+      if ((fs >> k) & 1u)
+        xp = !p.init ? 0.0f : (tl.few_rows ? w.iv : __ldg(p.init + tl.n0 + (tl.t0 + k) / p.T));
+      da[k] = ((w.f.term >> k) & 1u) ? 0.0f : g[k] * xp;
+      if (p.dinit && ((fs >> k) & 1u))
+        p.dinit[tl.n0 + (tl.t0 + k) / p.T] = ((w.f.term >> k) & 1u) ? 0.0f : w.a[k] * g[k];
+    }
+    if (p.da) st8(p.da, tl, da);
+  }
+};
+
 }  // namespace rlscan

@@ -723,6 +723,40 @@ rlscan_status rlscan_affine_scan(const float *a, const float *b, const uint8_t *
   return reverse ? go(AffineOp<true>{}) : go(AffineOp<false>{});
 }
 
+rlscan_status rlscan_affine_scan_grad(const float *a, const float *x, const float *dy, const uint8_t *reset,
+                                      const float *init, float *da, float *db, float *dinit, int64_t N,
+                                      int64_t T, int32_t reverse, rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1) || (reverse != 0 && reverse != 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(a), c.need(x), c.need(dy), c.need(db);
+  c.input(a, nt * 4, 4), c.input(x, nt * 4, 4), c.input(dy, nt * 4, 4), c.input(reset, nt, 1);
+  c.input(init, size_t(N) * 4, 4);
+  c.output(db, nt * 4, 4), c.output(da, nt * 4, 4), c.output(dinit, size_t(N) * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  const Plan pl = make_plan(RLSCAN_EST_AFFINE_SCAN_GRAD, N, T, 1);
+  auto vec = [&](int64_t r0) {
+    const int64_t o = r0 * T;
+    return aligned(adv(a, o), 32) && aligned(adv(x, o), 32) && aligned(adv(dy, o), 32) &&
+           aligned(adv(db, o), 32) && aligned(adv(da, o), 32) && aligned(adv(reset, o), 8);
+  };
+  auto go = [&](auto op) {
+    using Op = decltype(op);
+    return run<Op>(
+        pl, N, T, stream,
+        [&](int64_t r0) {
+          const int64_t o = r0 * T;
+          return typename Op::Args{adv(a, o),     adv(x, o),  adv(dy, o),    adv(init, r0), adv(reset, o),
+                                   nullptr,        adv(da, o), adv(db, o),    adv(dinit, r0), uint32_t(T)};
+        },
+        vec);
+  };
+  return reverse ? go(AffineGradOp<true>{}) : go(AffineGradOp<false>{});
+}
+
 rlscan_status rlscan_sync_status(rlscan_stream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) {
     cudaGetLastError();
@@ -788,7 +822,7 @@ int rlscan_abi_version(void) { return RLSCAN_ABI_VERSION; }
 
 rlscan_status rlscan_query_plan(rlscan_estimator est, int64_t N, int64_t T, int64_t A,
                                 rlscan_plan_info *info) {
-  if (!info || int(est) < 0 || int(est) > int(RLSCAN_EST_AFFINE_SCAN)) return RLSCAN_ERR_INVALID_ARG;
+  if (!info || int(est) < 0 || int(est) > int(RLSCAN_EST_AFFINE_SCAN_GRAD)) return RLSCAN_ERR_INVALID_ARG;
   if (est != RLSCAN_EST_RETRACE) A = 1;
   if (A < 1 || A > kMaxActions || !dims_ok(N, T, A)) return RLSCAN_ERR_INVALID_ARG;
   std::memset(info, 0, sizeof(*info));

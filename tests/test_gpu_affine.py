@@ -129,3 +129,53 @@ def test_affine_reset_everywhere_returns_b():
         got, _ = run_both(d, reverse)
         np.testing.assert_array_equal(got, d["b"].astype(np.float64))
 
+
+
+# --------------------------------------------------------------------------
+# gradient (adjoint) of the affine scan
+# --------------------------------------------------------------------------
+
+def run_grad(d, dy, reverse, device="cuda"):
+    x_ref = oracle.affine_scan(d["a"], d["b"], d["reset"], d["init"], reverse=reverse).astype(np.float32)
+    t = {k: None if v is None else torch.from_numpy(np.ascontiguousarray(v)).to(device)
+         for k, v in dict(d, x=x_ref, dy=dy).items()}
+    da, db, dinit = slr.rlscan_affine_scan_grad(t["a"], t["x"], t["dy"], t["reset"], t["init"], reverse=reverse)
+    rda, rdb, rdinit = oracle.affine_scan_grad(d["a"], x_ref, dy, d["reset"], d["init"], reverse=reverse)
+    return (da.cpu().numpy().astype(np.float64), db.cpu().numpy().astype(np.float64),
+            None if dinit is None else dinit.cpu().numpy().astype(np.float64)), (rda, rdb, rdinit)
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("N,T", CASES)
+def test_affine_grad_matches_oracle(N, T, reverse):
+    d = synthetic.make_affine_inputs(N, T, seed=2700 + N + T, p_reset=0.01)
+    dy = np.random.default_rng(N + T).standard_normal((N, T)).astype(np.float32)
+    got, ref = run_grad(d, dy, reverse)
+    for name, g, r in zip(("da", "db", "dinit"), got, ref):
+        assert_close(g, r, f"{name} N={N} T={T} reverse={reverse}")
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("block", [128, 256, 512])
+@pytest.mark.parametrize("lookback", [0, 1])
+def test_affine_grad_every_plan(reverse, block, lookback, options):
+    options("force_block", block)
+    options("force_lookback", lookback)
+    for N, T in ((100, 100), (3, 9000), (17, 1537), (9, 5)):
+        d = synthetic.make_affine_inputs(N, T, seed=2800 + N, p_reset=0.02)
+        dy = np.random.default_rng(T).standard_normal((N, T)).astype(np.float32)
+        got, ref = run_grad(d, dy, reverse)
+        for name, g, r in zip(("da", "db", "dinit"), got, ref):
+            assert_close(g, r, f"{name} block={block} lookback={lookback} N={N} T={T}")
+
+
+def test_affine_grad_optional_outputs_and_host_tensors():
+    d = synthetic.make_affine_inputs(12, 333, seed=2901, p_reset=0.03, with_init=False)
+    dy = np.random.default_rng(7).standard_normal((12, 333)).astype(np.float32)
+    x = oracle.affine_scan(d["a"], d["b"], d["reset"], None, reverse=True).astype(np.float32)
+    t = {k: torch.from_numpy(v) if v is not None else None for k, v in dict(d, x=x, dy=dy).items()}
+    da, db, dinit = slr.rlscan_affine_scan_grad(t["a"], t["x"], t["dy"], t["reset"], None, reverse=True,
+                                                need_da=False, need_dinit=False)
+    assert da is None and dinit is None
+    _, rdb, _ = oracle.affine_scan_grad(d["a"], x, dy, d["reset"], None, reverse=True)
+    assert_close(db.numpy().astype(np.float64), rdb, "db only, host tensors")

@@ -233,6 +233,19 @@ rlscan_status rlscan_affine_scan(const float *a, const float *b, const uint8_t *
                                  float *x, int64_t N, int64_t T, int32_t reverse, rlscan_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * rlscan_affine_scan with bfloat16 storage (bf16 I/O): a, b, init and x hold
+ * bfloat16 values (IEEE binary32 truncated to its top 16 bits, passed as
+ * uint16_t), reset is uint8 as above.  Arithmetic is fp32 in registers; each
+ * x_t is rounded to bf16 (round to nearest, ties to even; 8 significant
+ * bits) when stored, so |x - exact| <= 2^-8 |x| plus the fp32 error.  Half
+ * the bytes of the fp32
+ * call.  Vectorised when a, b and x are 16-byte aligned.
+ * ------------------------------------------------------------------------- */
+rlscan_status rlscan_affine_scan_bf16(const uint16_t *a, const uint16_t *b, const uint8_t *reset,
+                                      const uint16_t *init, uint16_t *x, int64_t N, int64_t T, int32_t reverse,
+                                      rlscan_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Gradient of rlscan_affine_scan (its adjoint), for a loss L whose direct
  * derivative with respect to x_t is dy_t.  `x` is the forward call's output
  * and `reverse` its direction.  The chain rule through the recurrence is an
@@ -284,7 +297,8 @@ typedef enum rlscan_estimator {
   RLSCAN_EST_ELIG_TRACE = 5,
   RLSCAN_EST_EPISODIC_PREFIX_SUM = 6,
   RLSCAN_EST_AFFINE_SCAN = 7,
-  RLSCAN_EST_AFFINE_SCAN_GRAD = 8
+  RLSCAN_EST_AFFINE_SCAN_GRAD = 8,
+  RLSCAN_EST_AFFINE_SCAN_BF16 = 9
 } rlscan_estimator;
 
 /* How a call of the given shape is executed (no device work, no allocation). */

@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "RlscanError", "lib", "rlscan_gae", "rlscan_vtrace", "rlscan_retrace", "rlscan_td_lambda",
     "rlscan_discounted_return", "rlscan_elig_trace", "rlscan_episodic_prefix_sum",
-    "rlscan_affine_scan", "rlscan_affine_scan_grad", "rlscan_sync_status", "rlscan_status_string", "rlscan_release_workspaces",
+    "rlscan_affine_scan", "rlscan_affine_scan_grad", "rlscan_affine_scan_bf16", "rlscan_sync_status", "rlscan_status_string", "rlscan_release_workspaces",
     "rlscan_abi_version", "rlscan_query_plan", "rlscan_set_option", "rlscan_get_option",
     "rlscan_reserve_workspace",
     "STATUS", "OPTIONS", "ESTIMATOR_IDS", "LIB_PATH",
@@ -36,7 +36,8 @@ STATUS = {0: "RLSCAN_OK", 1: "RLSCAN_ERR_INVALID_ARG", 2: "RLSCAN_ERR_OVERLAP",
 OPTIONS = {"lookback_timeout_ns": 1, "force_lookback": 2, "force_block": 3, "force_scalar": 4,
            "check_pointers": 5, "test_starve_lookback": 6, "pdl": 7}
 ESTIMATOR_IDS = {"gae": 0, "vtrace": 1, "retrace": 2, "td_lambda": 3, "discounted_return": 4,
-                 "elig_trace": 5, "episodic_prefix_sum": 6, "affine_scan": 7, "affine_scan_grad": 8}
+                 "elig_trace": 5, "episodic_prefix_sum": 6, "affine_scan": 7, "affine_scan_grad": 8,
+                 "affine_scan_bf16": 9}
 
 
 class RlscanError(RuntimeError):
@@ -63,6 +64,7 @@ _SIGNATURES = {
     "rlscan_episodic_prefix_sum": [_VP] * 4 + [_I64, _I64, _VP],
     "rlscan_affine_scan": [_VP] * 5 + [_I64, _I64, ctypes.c_int32, _VP],
     "rlscan_affine_scan_grad": [_VP] * 8 + [_I64, _I64, ctypes.c_int32, _VP],
+    "rlscan_affine_scan_bf16": [_VP] * 5 + [_I64, _I64, ctypes.c_int32, _VP],
     "rlscan_sync_status": [_VP],
     "rlscan_release_workspaces": [],
     "rlscan_reserve_workspace": [_I64, _VP],
@@ -320,6 +322,21 @@ def rlscan_affine_scan(a, b, reset=None, init=None, *, reverse=False, x=None, st
     out = c.output(x, torch.float32, (N, T), "x")
     st = lib().rlscan_affine_scan(c.ptr(aa), c.ptr(bb), c.ptr(rs), c.ptr(x0), c.ptr(out), N, T,
                                   1 if reverse else 0, c.stream(stream))
+    return c.finish(st, (out,))[0]
+
+
+def rlscan_affine_scan_bf16(a, b, reset=None, init=None, *, reverse=False, x=None, stream=None):
+    """rlscan_affine_scan on bfloat16 tensors (fp32 arithmetic, bf16 result).
+    Returns the [N, T] bfloat16 x."""
+    N, T = _nt(a, "rlscan_affine_scan_bf16")
+    c = _Call("rlscan_affine_scan_bf16", a)
+    aa = c.tensor(a, torch.bfloat16, (N, T), "a")
+    bb = c.tensor(b, torch.bfloat16, (N, T), "b")
+    rs = c.tensor(reset, torch.uint8, (N, T), "reset", required=False)
+    x0 = c.tensor(init, torch.bfloat16, (N,), "init", required=False)
+    out = c.output(x, torch.bfloat16, (N, T), "x")
+    st = lib().rlscan_affine_scan_bf16(c.ptr(aa), c.ptr(bb), c.ptr(rs), c.ptr(x0), c.ptr(out), N, T,
+                                       1 if reverse else 0, c.stream(stream))
     return c.finish(st, (out,))[0]
 
 

@@ -31,6 +31,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "scan_core.cuh"
@@ -125,13 +126,55 @@ __device__ __forceinline__ void st8(int32_t *p, const Tile &tl, const uint32_t (
   }
 }
 
+// bf16 storage (bf16 I/O): 8 steps are 16 bytes, one 128-bit access; values
+// widen to fp32 exactly (the bf16 bits are the top half of the fp32 bits) and
+// narrow with round-to-nearest-even.
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+__device__ __forceinline__ void ld8(const __nv_bfloat16 *p, const Tile &tl, float (&v)[8]) {
+  if (tl.fast) {
+    uint32_t u[4];
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
+                 : "l"(p + tl.i0));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = bf16_lo(u[j]);
+      v[2 * j + 1] = bf16_hi(u[j]);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = k < tl.nvalid ? __bfloat162float(__ldg(p + tl.i0 + k)) : 0.0f;
+  }
+}
+__device__ __forceinline__ void st8(__nv_bfloat16 *p, const Tile &tl, const float (&v)[8]) {
+  if (tl.full) {
+    uint32_t u[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+      u[j] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p + tl.i0), "r"(u[0]), "r"(u[1]), "r"(u[2]),
+                 "r"(u[3])
+                 : "memory");
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if ((tl.valid >> k) & 1u) p[tl.i0 + k] = __float2bfloat16_rn(v[k]);
+  }
+}
+__device__ __forceinline__ float ld1(const float *p) { return __ldg(p); }
+__device__ __forceinline__ float ld1(const __nv_bfloat16 *p) { return __bfloat162float(__ldg(p)); }
+
 // Per-row value (bootstrap / initial trace) of the tile's row edge, issued
 // with the tile's other loads: its address follows from the tile position.
 // Tiles of rows shorter than 8 steps (several edges) load theirs in coef().
-__device__ __forceinline__ float edge_value(const float *src, const Tile &tl, const FastDiv &fd) {
+template <class E>
+__device__ __forceinline__ float edge_value(const E *src, const Tile &tl, const FastDiv &fd) {
   if (src == nullptr || !tl.few_rows || tl.edge == 0u) return 0.0f;
   const uint32_t k = __ffs(tl.edge) - 1u;
-  return __ldg(src + tl.n0 + fd.div(tl.t0 + k));
+  return ld1(src + tl.n0 + fd.div(tl.t0 + k));
 }
 
 // Terminated / truncated masks of a tile (bit k: step k).
@@ -476,15 +519,15 @@ struct PrefixSumOp {
 // b + a init (init NULL: 0).  The reset flags travel in the flag slot of
 // `term`; `trunc` is NULL.
 // ---------------------------------------------------------------------------
-template <bool BWD>
+template <bool BWD, class E = float>
 struct AffineOp {
   static constexpr int kRegs = 40, kRegsLookback = 40;  // registers per thread, chosen by measurement
   using V = float;
   static constexpr bool kBackward = BWD;
   struct Args {
-    const float *a, *b, *init;
+    const E *a, *b, *init;        // E: float, or __nv_bfloat16 for bf16 I/O (fp32 arithmetic)
     const uint8_t *term, *trunc;  // term: reset flags (nullable); trunc: NULL
-    float *out;
+    E *out;
   };
   struct Raw {
     float a[8], b[8];
@@ -509,7 +552,7 @@ struct AffineOp {
     for (int k = 0; k < 8; ++k) {
       float b = w.b[k];
       if (((init_at >> k) & 1u) && p.init)
-        b = fmaf(w.a[k], tl.few_rows ? w.ev : __ldg(p.init + tl.n0 + fd.div(tl.t0 + k)), b);
+        b = fmaf(w.a[k], tl.few_rows ? w.ev : ld1(p.init + tl.n0 + fd.div(tl.t0 + k)), b);
       c[k] = Aff<float>{((cut >> k) & 1u) ? 0.0f : w.a[k], b};
     }
   }

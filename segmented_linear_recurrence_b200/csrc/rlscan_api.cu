@@ -723,6 +723,41 @@ rlscan_status rlscan_affine_scan(const float *a, const float *b, const uint8_t *
   return reverse ? go(AffineOp<true>{}) : go(AffineOp<false>{});
 }
 
+rlscan_status rlscan_affine_scan_bf16(const uint16_t *a, const uint16_t *b, const uint8_t *reset,
+                                      const uint16_t *init, uint16_t *x, int64_t N, int64_t T, int32_t reverse,
+                                      rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1) || (reverse != 0 && reverse != 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(a), c.need(b), c.need(x);
+  c.input(a, nt * 2, 2), c.input(b, nt * 2, 2), c.input(reset, nt, 1), c.input(init, size_t(N) * 2, 2);
+  c.output(x, nt * 2, 2);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  const Plan pl = make_plan(RLSCAN_EST_AFFINE_SCAN_BF16, N, T, 1);
+  using B16 = __nv_bfloat16;
+  const B16 *ab = reinterpret_cast<const B16 *>(a), *bb = reinterpret_cast<const B16 *>(b);
+  const B16 *ib = reinterpret_cast<const B16 *>(init);
+  B16 *xb = reinterpret_cast<B16 *>(x);
+  auto vec = [&](int64_t r0) {
+    const int64_t o = r0 * T;
+    return aligned(adv(ab, o), 16) && aligned(adv(bb, o), 16) && aligned(adv(xb, o), 16) && aligned(adv(reset, o), 8);
+  };
+  auto go = [&](auto op) {
+    using Op = decltype(op);
+    return run<Op>(
+        pl, N, T, stream,
+        [&](int64_t r0) {
+          const int64_t o = r0 * T;
+          return typename Op::Args{adv(ab, o), adv(bb, o), adv(ib, r0), adv(reset, o), nullptr, adv(xb, o)};
+        },
+        vec);
+  };
+  return reverse ? go(AffineOp<true, B16>{}) : go(AffineOp<false, B16>{});
+}
+
 rlscan_status rlscan_affine_scan_grad(const float *a, const float *x, const float *dy, const uint8_t *reset,
                                       const float *init, float *da, float *db, float *dinit, int64_t N,
                                       int64_t T, int32_t reverse, rlscan_stream_t stream) {
@@ -822,7 +857,7 @@ int rlscan_abi_version(void) { return RLSCAN_ABI_VERSION; }
 
 rlscan_status rlscan_query_plan(rlscan_estimator est, int64_t N, int64_t T, int64_t A,
                                 rlscan_plan_info *info) {
-  if (!info || int(est) < 0 || int(est) > int(RLSCAN_EST_AFFINE_SCAN_GRAD)) return RLSCAN_ERR_INVALID_ARG;
+  if (!info || int(est) < 0 || int(est) > int(RLSCAN_EST_AFFINE_SCAN_BF16)) return RLSCAN_ERR_INVALID_ARG;
   if (est != RLSCAN_EST_RETRACE) A = 1;
   if (A < 1 || A > kMaxActions || !dims_ok(N, T, A)) return RLSCAN_ERR_INVALID_ARG;
   std::memset(info, 0, sizeof(*info));

@@ -198,3 +198,11 @@ def test_affine_scan_argument_checks(L):
     p = slr.rlscan_query_plan("affine_scan", 4096, 2000)
     assert p["lookback"] == 0 and p["chunk_steps"] % 2000 == 0
     assert slr.rlscan_query_plan("affine_scan", 2, 100000)["lookback"] == 1
+
+
+def test_affine_scan_bf16_argument_checks(L):
+    a, b, x = P(BASE), P(BASE + 0x10000), P(BASE + 0x20000)
+    assert L.rlscan_affine_scan_bf16(a, b, None, None, x, 4, 8, 3, None) == INVALID  # direction
+    assert L.rlscan_affine_scan_bf16(a, b, None, None, P(BASE + 0x20001), 4, 8, 0, None) == INVALID  # odd address
+    assert L.rlscan_affine_scan_bf16(a, b, None, None, b, 4, 8, 0, None) == OVERLAP
+    assert slr.rlscan_query_plan("affine_scan_bf16", 4096, 2048)["lookback"] == 0

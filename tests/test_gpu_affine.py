@@ -179,3 +179,57 @@ def test_affine_grad_optional_outputs_and_host_tensors():
     assert da is None and dinit is None
     _, rdb, _ = oracle.affine_scan_grad(d["a"], x, dy, d["reset"], None, reverse=True)
     assert_close(db.numpy().astype(np.float64), rdb, "db only, host tensors")
+
+
+# --------------------------------------------------------------------------
+# bf16 I/O (rlscan_affine_scan_bf16): the oracle runs on the same bf16 values
+# widened to fp32 (exact); the result is fp32 arithmetic rounded to bf16 (8
+# significant bits: rounding to nearest is off by at most 2^-8 relative), so
+# |gpu - ref| <= 2^-8 |ref| + 1.1e-4 (1 + |ref|)
+# --------------------------------------------------------------------------
+
+def run_bf16(d, reverse, device="cuda"):
+    to16 = lambda v: None if v is None else torch.from_numpy(np.ascontiguousarray(v)).to(torch.bfloat16)  # noqa: E731
+    a16, b16, i16 = to16(d["a"]), to16(d["b"]), to16(d["init"])
+    rs = None if d["reset"] is None else torch.from_numpy(d["reset"])
+    mv = lambda t: None if t is None else t.to(device)  # noqa: E731
+    got = slr.rlscan_affine_scan_bf16(mv(a16), mv(b16), mv(rs), mv(i16), reverse=reverse)
+    f32 = lambda t: None if t is None else t.float().numpy()  # noqa: E731
+    ref = oracle.affine_scan(f32(a16), f32(b16), d["reset"], f32(i16), reverse=reverse)
+    return got.float().cpu().numpy().astype(np.float64), ref
+
+
+def assert_close_bf16(got, ref, what):
+    bound = 2.0 ** -8 * np.abs(ref) + 1.1e-4 * (1.0 + np.abs(ref))
+    bad = np.argwhere(np.abs(got - ref) > bound)
+    assert bad.size == 0, f"{what}: {bad.shape[0]} elements off, first {tuple(bad[0])}: " \
+                          f"gpu {got[tuple(bad[0])]} ref {ref[tuple(bad[0])]}"
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("N,T", CASES)
+def test_affine_bf16_matches_oracle(N, T, reverse):
+    d = synthetic.make_affine_inputs(N, T, seed=3000 + N + T, p_reset=0.01)
+    got, ref = run_bf16(d, reverse)
+    assert_close_bf16(got, ref, f"bf16 N={N} T={T} reverse={reverse}")
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("block", [128, 256, 512])
+@pytest.mark.parametrize("lookback", [0, 1])
+def test_affine_bf16_every_plan(reverse, block, lookback, options):
+    options("force_block", block)
+    options("force_lookback", lookback)
+    for N, T in ((100, 100), (3, 9000), (17, 1537)):
+        d = synthetic.make_affine_inputs(N, T, seed=3100 + N, p_reset=0.01)
+        got, ref = run_bf16(d, reverse)
+        assert_close_bf16(got, ref, f"bf16 block={block} lookback={lookback} N={N} T={T}")
+
+
+def test_affine_bf16_scalar_path_and_host_tensors(options):
+    d = synthetic.make_affine_inputs(11, 333, seed=3201, p_reset=0.02)
+    got, ref = run_bf16(d, True, device="cpu")
+    assert_close_bf16(got, ref, "bf16 host tensors")
+    options("force_scalar", 1)
+    got, ref = run_bf16(d, False)
+    assert_close_bf16(got, ref, "bf16 scalar path")

@@ -11,8 +11,9 @@
 // of the same page: termination -> successor value 0, truncation ->
 // trunc_value, window end -> bootstrap, counted once in the local term.
 //
-// A thread owns a tile of K = 8 consecutive steps: one 256-bit load per fp32
-// array, one 64-bit load per flag array.  Interface used by scan_kernel.cuh
+// A thread owns a tile of K consecutive steps (K = 8, or 16 where measured
+// faster): one 256-bit load per 8 steps of an fp32 array, one 64-bit load per
+// 8 flag bytes.  Interface used by scan_kernel.cuh
 // (all members static __device__):
 //   V, kBackward, Args, Raw
 //   load(args, tile, fd, lane, total, flags, raw)   given the tile's
@@ -38,45 +39,52 @@
 
 namespace rlscan {
 
-constexpr int kTile = 8;  // consecutive steps per thread
+constexpr int kTile = 8;  // default steps per thread; an estimator may use 16 (Op::K)
 
-// Geometry of one thread's tile.
+// Geometry of one thread's tile of K consecutive steps (K = 8 or 16).
 struct Tile {
-  uint32_t i0;     // first step (flat, launch-local; a multiple of 8)
-  int nvalid;      // steps of the tile inside the launch (0..8): these may be loaded
+  uint32_t i0;     // first step (flat, launch-local; a multiple of K)
+  int nvalid;      // steps of the tile inside the launch (0..K): these may be loaded
   uint32_t valid;  // bit k: step k belongs to this block (scanned and stored)
   uint32_t n0, t0; // row and time of step i0
   uint32_t edge;   // bit k: step k is on its row's dependency edge
                    //   (backward: t = T-1, forward: t = 0)
   bool fast;       // 256-bit (flags: 64-bit) loads allowed
-  bool full;       // ... and all 8 steps are the block's: 256-bit stores
-  bool few_rows;   // T >= 8: at most one row edge in the tile
+  bool full;       // ... and all K steps are the block's: 256-bit stores
+  bool few_rows;   // T >= K: at most one row edge in the tile
 };
 
 // ---------------------------------------------------------------------------
-// loads / stores of 8 consecutive steps
+// loads / stores of a tile: 8 steps per 256-bit access (flags: 64-bit)
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void ld8(const float *p, const Tile &tl, float (&v)[8]) {
+__device__ __forceinline__ void ld8_raw(const float *a, float *v) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+               : "l"(a));
+}
+__device__ __forceinline__ void ld8_raw(const int32_t *a, uint32_t *v) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "l"(a));
+}
+template <int K>
+__device__ __forceinline__ void ld_tile(const float *p, const Tile &tl, float (&v)[K]) {
   if (tl.fast) {
-    asm volatile("ld.global.nc.L1::no_allocate.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]),
-                   "=f"(v[7])
-                 : "l"(p + tl.i0));
+#pragma unroll
+    for (int j = 0; j < K / 8; ++j) ld8_raw(p + tl.i0 + 8 * j, &v[8 * j]);
   } else {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = k < tl.nvalid ? __ldg(p + tl.i0 + k) : 0.0f;
+    for (int k = 0; k < K; ++k) v[k] = k < tl.nvalid ? __ldg(p + tl.i0 + k) : 0.0f;
   }
 }
-
-__device__ __forceinline__ void ld8(const int32_t *p, const Tile &tl, uint32_t (&v)[8]) {
+template <int K>
+__device__ __forceinline__ void ld_tile(const int32_t *p, const Tile &tl, uint32_t (&v)[K]) {
   if (tl.fast) {
-    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-                   "=r"(v[7])
-                 : "l"(p + tl.i0));
+#pragma unroll
+    for (int j = 0; j < K / 8; ++j) ld8_raw(p + tl.i0 + 8 * j, &v[8 * j]);
   } else {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = k < tl.nvalid ? uint32_t(__ldg(p + tl.i0 + k)) : 0u;
+    for (int k = 0; k < K; ++k) v[k] = k < tl.nvalid ? uint32_t(__ldg(p + tl.i0 + k)) : 0u;
   }
 }
 
@@ -88,40 +96,56 @@ __device__ __forceinline__ uint32_t nonzero_bytes4(uint32_t w) {
   const uint32_t hi = (((w & 0x7f7f7f7fu) + 0x7f7f7f7fu) | w) & 0x80808080u;
   return (hi * 0x00204081u) >> 28;
 }
-__device__ __forceinline__ uint32_t ld8_flags(const uint8_t *p, const Tile &tl) {
+template <int K>
+__device__ __forceinline__ uint32_t ld_flags(const uint8_t *p, const Tile &tl) {
   if (p == nullptr) return 0u;
-  if (tl.fast) {
-    uint32_t lo, hi;
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(lo), "=r"(hi) : "l"(p + tl.i0));
-    return nonzero_bytes4(lo) | (nonzero_bytes4(hi) << 4);
-  }
   uint32_t m = 0;
+  if (tl.fast) {
 #pragma unroll
-  for (int k = 0; k < 8; ++k)
+    for (int j = 0; j < K / 8; ++j) {
+      uint32_t lo, hi;
+      asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                   : "=r"(lo), "=r"(hi)
+                   : "l"(p + tl.i0 + 8 * j));
+      m |= (nonzero_bytes4(lo) | (nonzero_bytes4(hi) << 4)) << (8 * j);
+    }
+    return m;
+  }
+#pragma unroll
+  for (int k = 0; k < K; ++k)
     if (k < tl.nvalid && __ldg(p + tl.i0 + k) != 0) m |= 1u << k;
   return m;
 }
 
-__device__ __forceinline__ void st8(float *p, const Tile &tl, const float (&v)[8]) {
+__device__ __forceinline__ void st8_raw(float *a, const float *v) {
+  asm volatile("st.global.cs.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(a), "f"(v[0]), "f"(v[1]), "f"(v[2]),
+               "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+               : "memory");
+}
+__device__ __forceinline__ void st8_raw(int32_t *a, const uint32_t *v) {
+  asm volatile("st.global.cs.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(a), "r"(v[0]), "r"(v[1]), "r"(v[2]),
+               "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+template <int K>
+__device__ __forceinline__ void st_tile(float *p, const Tile &tl, const float (&v)[K]) {
   if (tl.full) {
-    asm volatile("st.global.cs.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p + tl.i0), "f"(v[0]), "f"(v[1]),
-                 "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
-                 : "memory");
+#pragma unroll
+    for (int j = 0; j < K / 8; ++j) st8_raw(p + tl.i0 + 8 * j, &v[8 * j]);
   } else {
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < K; ++k)
       if ((tl.valid >> k) & 1u) p[tl.i0 + k] = v[k];
   }
 }
-
-__device__ __forceinline__ void st8(int32_t *p, const Tile &tl, const uint32_t (&v)[8]) {
+template <int K>
+__device__ __forceinline__ void st_tile(int32_t *p, const Tile &tl, const uint32_t (&v)[K]) {
   if (tl.full) {
-    asm volatile("st.global.cs.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p + tl.i0), "r"(v[0]), "r"(v[1]),
-                 "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-                 : "memory");
+#pragma unroll
+    for (int j = 0; j < K / 8; ++j) st8_raw(p + tl.i0 + 8 * j, &v[8 * j]);
   } else {
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < K; ++k)
       if ((tl.valid >> k) & 1u) p[tl.i0 + k] = int32_t(v[k]);
   }
 }
@@ -131,36 +155,44 @@ __device__ __forceinline__ void st8(int32_t *p, const Tile &tl, const uint32_t (
 // narrow with round-to-nearest-even.
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
-__device__ __forceinline__ void ld8(const __nv_bfloat16 *p, const Tile &tl, float (&v)[8]) {
+template <int K>
+__device__ __forceinline__ void ld_tile(const __nv_bfloat16 *p, const Tile &tl, float (&v)[K]) {
   if (tl.fast) {
-    uint32_t u[4];
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
-                 : "l"(p + tl.i0));
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      v[2 * j] = bf16_lo(u[j]);
-      v[2 * j + 1] = bf16_hi(u[j]);
+    for (int q = 0; q < K / 8; ++q) {
+      uint32_t u[4];
+      asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
+                   : "l"(p + tl.i0 + 8 * q));
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[8 * q + 2 * j] = bf16_lo(u[j]);
+        v[8 * q + 2 * j + 1] = bf16_hi(u[j]);
+      }
     }
   } else {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = k < tl.nvalid ? __bfloat162float(__ldg(p + tl.i0 + k)) : 0.0f;
+    for (int k = 0; k < K; ++k) v[k] = k < tl.nvalid ? __bfloat162float(__ldg(p + tl.i0 + k)) : 0.0f;
   }
 }
-__device__ __forceinline__ void st8(__nv_bfloat16 *p, const Tile &tl, const float (&v)[8]) {
+template <int K>
+__device__ __forceinline__ void st_tile(__nv_bfloat16 *p, const Tile &tl, const float (&v)[K]) {
   if (tl.full) {
-    uint32_t u[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
-      u[j] = *reinterpret_cast<const uint32_t *>(&h);
+    for (int q = 0; q < K / 8; ++q) {
+      uint32_t u[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * q + 2 * j], v[8 * q + 2 * j + 1]);
+        u[j] = *reinterpret_cast<const uint32_t *>(&h);
+      }
+      asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p + tl.i0 + 8 * q), "r"(u[0]), "r"(u[1]),
+                   "r"(u[2]), "r"(u[3])
+                   : "memory");
     }
-    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p + tl.i0), "r"(u[0]), "r"(u[1]), "r"(u[2]),
-                 "r"(u[3])
-                 : "memory");
   } else {
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < K; ++k)
       if ((tl.valid >> k) & 1u) p[tl.i0 + k] = __float2bfloat16_rn(v[k]);
   }
 }
@@ -169,7 +201,7 @@ __device__ __forceinline__ float ld1(const __nv_bfloat16 *p) { return __bfloat16
 
 // Per-row value (bootstrap / initial trace) of the tile's row edge, issued
 // with the tile's other loads: its address follows from the tile position.
-// Tiles of rows shorter than 8 steps (several edges) load theirs in coef().
+// Tiles of rows shorter than K steps (several edges) load theirs in coef().
 template <class E>
 __device__ __forceinline__ float edge_value(const E *src, const Tile &tl, const FastDiv &fd) {
   if (src == nullptr || !tl.few_rows || tl.edge == 0u) return 0.0f;
@@ -187,20 +219,21 @@ struct Flags {
 // row's bootstrap at a row end (`boot` may be NULL: 0); termination wins over
 // truncation, and both over the row end.  trunc_value is the only load whose
 // address depends on loaded data; warps without a truncated step skip it.
+template <int K>
 __device__ __forceinline__ void boundary_successors(const float *tv, const float *boot, float ev, const Tile &tl,
-                                                    Flags f, const FastDiv &fd, float (&bv)[8]) {
+                                                    Flags f, const FastDiv &fd, float (&bv)[K]) {
   const uint32_t tr = f.trunc & ~f.term & tl.valid;
   const uint32_t ed = tl.edge & ~f.term & ~f.trunc;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) bv[k] = 0.0f;
+  for (int k = 0; k < K; ++k) bv[k] = 0.0f;
   if (__any_sync(0xffffffffu, tr != 0u)) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < K; ++k)
       if ((tr >> k) & 1u) bv[k] = __ldg(tv + tl.i0 + k);
   }
   if (ed != 0u) {  // at most one row end per tile when T >= 8
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < K; ++k)
       if ((ed >> k) & 1u) bv[k] = tl.few_rows ? ev : (boot ? __ldg(boot + tl.n0 + fd.div(tl.t0 + k)) : 0.0f);
   }
 }
@@ -209,7 +242,9 @@ __device__ __forceinline__ void boundary_successors(const float *tv, const float
 // GAE (Schulman et al. 2016): x = advantage, a = gamma lambda cont,
 // b = r + gamma nv - v.  Outputs advantages = x, returns = x + v.
 // ---------------------------------------------------------------------------
-struct GaeOp {
+template <int K_ = kTile>
+struct GaeOpT {
+  static constexpr int K = K_;  // steps per thread
   static constexpr int kRegs = 48, kRegsLookback = 48;  // registers per thread, chosen by measurement
   using V = float;
   static constexpr bool kBackward = true;
@@ -220,17 +255,17 @@ struct GaeOp {
     float gamma, gl;
   };
   struct Raw {
-    float r[8], v[8], bv[8];  // bv: successor values at boundary steps
+    float r[K], v[K], bv[K];  // bv: successor values at boundary steps
     Flags f;
     float halo;  // v of the step after the tile (lane 31 only)
     float ev;    // bootstrap of the tile's row end
   };
   static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int lane,
                                               uint32_t total, Flags f, Raw &w) {
-    ld8(p.r, tl, w.r);
-    ld8(p.v, tl, w.v);
+    ld_tile(p.r, tl, w.r);
+    ld_tile(p.v, tl, w.v);
     w.f = f;
-    w.halo = (lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total) ? __ldg(p.v + tl.i0 + 8u) : 0.0f;
+    w.halo = (lane == 31 && tl.nvalid == K && tl.i0 + uint32_t(K) < total) ? __ldg(p.v + tl.i0 + uint32_t(K)) : 0.0f;
     w.ev = edge_value(p.boot, tl, fd);
   }
   static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w) {
@@ -239,33 +274,36 @@ struct GaeOp {
   static __device__ __forceinline__ float nbr_of(const Raw &w) { return w.v[0]; }
   static __device__ __forceinline__ float halo_of(const Raw &w) { return w.halo; }
   static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w,
-                                              float next7, Aff<float> (&c)[8]) {
+                                              float next7, Aff<float> (&c)[K]) {
     const uint32_t special = w.f.term | w.f.trunc | tl.edge;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < K; ++k) {
       const bool sp = (special >> k) & 1u;
-      const float next = k < 7 ? w.v[k < 7 ? k + 1 : 7] : next7;
+      const float next = k < K - 1 ? w.v[k < K - 1 ? k + 1 : K - 1] : next7;
       const float nv = sp ? w.bv[k] : next;
       c[k] = Aff<float>{sp ? 0.0f : p.gl, fmaf(p.gamma, nv, w.r[k]) - w.v[k]};
     }
   }
-  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &w, const Aff<float> (&)[8],
-                                              const float (&x)[8], const float (&)[8]) {
-    st8(p.adv, tl, x);
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &w, const Aff<float> (&)[K],
+                                              const float (&x)[K], const float (&)[K]) {
+    st_tile(p.adv, tl, x);
     if (p.ret) {
-      float ret[8];
+      float ret[K];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) ret[k] = x[k] + w.v[k];
-      st8(p.ret, tl, ret);
+      for (int k = 0; k < K; ++k) ret[k] = x[k] + w.v[k];
+      st_tile(p.ret, tl, ret);
     }
   }
 };
+using GaeOp = GaeOpT<>;
 
 // ---------------------------------------------------------------------------
 // TD(lambda) returns: a = gamma lambda cont, b = r + gamma (1 - lambda) v_{t+1}
 // inside an episode, b = r + gamma nv at a boundary.  Output x.
 // ---------------------------------------------------------------------------
-struct TdLambdaOp {
+template <int K_ = kTile>
+struct TdLambdaOpT {
+  static constexpr int K = K_;  // steps per thread
   static constexpr int kRegs = 48, kRegsLookback = 48;  // registers per thread, chosen by measurement
   using V = float;
   static constexpr bool kBackward = true;
@@ -276,16 +314,16 @@ struct TdLambdaOp {
     float gamma, gl, g1l;  // gamma, gamma*lambda, gamma*(1-lambda)
   };
   struct Raw {
-    float r[8], v[8], bv[8];
+    float r[K], v[K], bv[K];
     Flags f;
     float halo, ev;
   };
   static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int lane,
                                               uint32_t total, Flags f, Raw &w) {
-    ld8(p.r, tl, w.r);
-    ld8(p.v, tl, w.v);
+    ld_tile(p.r, tl, w.r);
+    ld_tile(p.v, tl, w.v);
     w.f = f;
-    w.halo = (lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total) ? __ldg(p.v + tl.i0 + 8u) : 0.0f;
+    w.halo = (lane == 31 && tl.nvalid == K && tl.i0 + uint32_t(K) < total) ? __ldg(p.v + tl.i0 + uint32_t(K)) : 0.0f;
     w.ev = edge_value(p.boot, tl, fd);
   }
   static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w) {
@@ -294,26 +332,29 @@ struct TdLambdaOp {
   static __device__ __forceinline__ float nbr_of(const Raw &w) { return w.v[0]; }
   static __device__ __forceinline__ float halo_of(const Raw &w) { return w.halo; }
   static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w,
-                                              float next7, Aff<float> (&c)[8]) {
+                                              float next7, Aff<float> (&c)[K]) {
     const uint32_t special = w.f.term | w.f.trunc | tl.edge;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < K; ++k) {
       const bool sp = (special >> k) & 1u;
-      const float next = k < 7 ? w.v[k < 7 ? k + 1 : 7] : next7;
+      const float next = k < K - 1 ? w.v[k < K - 1 ? k + 1 : K - 1] : next7;
       c[k] = sp ? Aff<float>{0.0f, fmaf(p.gamma, w.bv[k], w.r[k])} : Aff<float>{p.gl, fmaf(p.g1l, next, w.r[k])};
     }
   }
-  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[8],
-                                              const float (&x)[8], const float (&)[8]) {
-    st8(p.out, tl, x);
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[K],
+                                              const float (&x)[K], const float (&)[K]) {
+    st_tile(p.out, tl, x);
   }
 };
+using TdLambdaOp = TdLambdaOpT<>;
 
 // ---------------------------------------------------------------------------
 // Discounted return: a = gamma cont, b = r (+ gamma nv at a boundary).
 // bootstrap may be NULL (zero at the window end).  Output x.
 // ---------------------------------------------------------------------------
-struct DiscountedOp {
+template <int K_ = kTile>
+struct DiscountedOpT {
+  static constexpr int K = K_;  // steps per thread
   static constexpr int kRegs = 32, kRegsLookback = 40;  // registers per thread, chosen by measurement
   using V = float;
   static constexpr bool kBackward = true;
@@ -324,13 +365,13 @@ struct DiscountedOp {
     float gamma;
   };
   struct Raw {
-    float r[8], bv[8];
+    float r[K], bv[K];
     Flags f;
     float ev;
   };
   static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int, uint32_t,
                                               Flags f, Raw &w) {
-    ld8(p.r, tl, w.r);
+    ld_tile(p.r, tl, w.r);
     w.f = f;
     w.ev = edge_value(p.boot, tl, fd);
   }
@@ -340,19 +381,20 @@ struct DiscountedOp {
   static __device__ __forceinline__ float nbr_of(const Raw &) { return 0.0f; }
   static __device__ __forceinline__ float halo_of(const Raw &) { return 0.0f; }
   static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w, float,
-                                              Aff<float> (&c)[8]) {
+                                              Aff<float> (&c)[K]) {
     const uint32_t special = w.f.term | w.f.trunc | tl.edge;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < K; ++k) {
       const bool sp = (special >> k) & 1u;
       c[k] = Aff<float>{sp ? 0.0f : p.gamma, fmaf(p.gamma, w.bv[k], w.r[k])};
     }
   }
-  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[8],
-                                              const float (&x)[8], const float (&)[8]) {
-    st8(p.out, tl, x);
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[K],
+                                              const float (&x)[K], const float (&)[K]) {
+    st_tile(p.out, tl, x);
   }
 };
+using DiscountedOp = DiscountedOpT<>;
 
 // ---------------------------------------------------------------------------
 // V-trace (Espeholt et al. 2018) with lambda-scaled traces, on d = vs - v:
@@ -361,7 +403,9 @@ struct DiscountedOp {
 // pg_adv = b + gamma rho cont x_{t+1}: rho (r + gamma vs_{t+1} - v) inside an
 // episode (vs_{t+1} = v_{t+1} + x_{t+1}), rho (r + gamma nv - v) at a boundary.
 // ---------------------------------------------------------------------------
-struct VtraceOp {
+template <int K_ = kTile>
+struct VtraceOpT {
+  static constexpr int K = K_;  // steps per thread
   static constexpr int kRegs = 56, kRegsLookback = 48;  // registers per thread, chosen by measurement
   using V = float;
   static constexpr bool kBackward = true;
@@ -372,17 +416,17 @@ struct VtraceOp {
     float gamma, lambda, rho_bar, c_bar;
   };
   struct Raw {
-    float lr[8], r[8], v[8], bv[8];  // coef() keeps gamma * rho * cont in lr for emit()
+    float lr[K], r[K], v[K], bv[K];  // coef() keeps gamma * rho * cont in lr for emit()
     Flags f;
     float halo, ev;
   };
   static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int lane,
                                               uint32_t total, Flags f, Raw &w) {
-    ld8(p.lr, tl, w.lr);
-    ld8(p.r, tl, w.r);
-    ld8(p.v, tl, w.v);
+    ld_tile(p.lr, tl, w.lr);
+    ld_tile(p.r, tl, w.r);
+    ld_tile(p.v, tl, w.v);
     w.f = f;
-    w.halo = (lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total) ? __ldg(p.v + tl.i0 + 8u) : 0.0f;
+    w.halo = (lane == 31 && tl.nvalid == K && tl.i0 + uint32_t(K) < total) ? __ldg(p.v + tl.i0 + uint32_t(K)) : 0.0f;
     w.ev = edge_value(p.boot, tl, fd);
   }
   static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w) {
@@ -391,12 +435,12 @@ struct VtraceOp {
   static __device__ __forceinline__ float nbr_of(const Raw &w) { return w.v[0]; }
   static __device__ __forceinline__ float halo_of(const Raw &w) { return w.halo; }
   static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w,
-                                              float next7, Aff<float> (&c)[8]) {
+                                              float next7, Aff<float> (&c)[K]) {
     const uint32_t special = w.f.term | w.f.trunc | tl.edge;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < K; ++k) {
       const bool sp = (special >> k) & 1u;
-      const float next = k < 7 ? w.v[k < 7 ? k + 1 : 7] : next7;
+      const float next = k < K - 1 ? w.v[k < K - 1 ? k + 1 : K - 1] : next7;
       const float nv = sp ? w.bv[k] : next;
       const float ratio = __expf(w.lr[k]);
       const float rho = fminf(p.rho_bar, ratio);
@@ -405,27 +449,30 @@ struct VtraceOp {
       w.lr[k] = sp ? 0.0f : p.gamma * rho;
     }
   }
-  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &w, const Aff<float> (&c)[8],
-                                              const float (&x)[8], const float (&xn)[8]) {
-    float o[8];
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &w, const Aff<float> (&c)[K],
+                                              const float (&x)[K], const float (&xn)[K]) {
+    float o[K];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) o[k] = x[k] + w.v[k];
-    st8(p.vs, tl, o);
+    for (int k = 0; k < K; ++k) o[k] = x[k] + w.v[k];
+    st_tile(p.vs, tl, o);
     if (p.pg) {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) o[k] = fmaf(w.lr[k], xn[k], c[k].b);
-      st8(p.pg, tl, o);
+      for (int k = 0; k < K; ++k) o[k] = fmaf(w.lr[k], xn[k], c[k].b);
+      st_tile(p.pg, tl, o);
     }
   }
 };
+using VtraceOp = VtraceOpT<>;
 
 // ---------------------------------------------------------------------------
 // Accumulating eligibility trace, forward: a = gamma lambda (1 - done_{t-1}),
 // b = g; the first step of a row folds in the carried-in trace:
 // b = g + gamma lambda init[n], a = 0.  Output x.
 // ---------------------------------------------------------------------------
-struct EligOp {
-  static constexpr int kRegs = 40, kRegsLookback = 32;  // registers per thread, chosen by measurement
+template <int K_ = kTile>
+struct EligOpT {
+  static constexpr int K = K_;  // steps per thread
+  static constexpr int kRegs = 56, kRegsLookback = 56;  // registers per thread, chosen by measurement
   using V = float;
   static constexpr bool kBackward = false;
   struct Args {
@@ -435,14 +482,14 @@ struct EligOp {
     float gl;
   };
   struct Raw {
-    float g[8];
+    float g[K];
     uint32_t done;  // bit k: step k terminated or truncated
     uint32_t halo;  // done flag of the step before the tile (lane 0 only)
     float ev;       // initial trace of the tile's row start
   };
   static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int lane, uint32_t,
                                               Flags f, Raw &w) {
-    ld8(p.g, tl, w.g);
+    ld_tile(p.g, tl, w.g);
     w.done = f.term | f.trunc;
     w.halo = 0u;
     if (lane == 0 && tl.i0 > 0u && tl.nvalid > 0)
@@ -450,31 +497,34 @@ struct EligOp {
     w.ev = edge_value(p.init, tl, fd);
   }
   static __device__ __forceinline__ void fetch_boundary(const Args &, const Tile &, const FastDiv &, Raw &) {}
-  static __device__ __forceinline__ uint32_t nbr_of(const Raw &w) { return (w.done >> 7) & 1u; }
+  static __device__ __forceinline__ uint32_t nbr_of(const Raw &w) { return (w.done >> (K - 1)) & 1u; }
   static __device__ __forceinline__ uint32_t halo_of(const Raw &w) { return w.halo; }
   static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w,
-                                              uint32_t prev7, Aff<float> (&c)[8]) {
-    const uint32_t cut = (((w.done << 1) | prev7) | tl.edge) & 0xffu;  // bit k: a_k = 0
+                                              uint32_t prev7, Aff<float> (&c)[K]) {
+    const uint32_t cut = (((w.done << 1) | prev7) | tl.edge) & ((1u << K) - 1u);  // bit k: a_k = 0
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < K; ++k) {
       float b = w.g[k];
       if (((tl.edge >> k) & 1u) && p.init)
         b = fmaf(p.gl, tl.few_rows ? w.ev : __ldg(p.init + tl.n0 + fd.div(tl.t0 + k)), b);
       c[k] = Aff<float>{((cut >> k) & 1u) ? 0.0f : p.gl, b};
     }
   }
-  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[8],
-                                              const float (&x)[8], const float (&)[8]) {
-    st8(p.out, tl, x);
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[K],
+                                              const float (&x)[K], const float (&)[K]) {
+    st_tile(p.out, tl, x);
   }
 };
+using EligOp = EligOpT<16>;  // 16 steps per thread: measured faster
 
 // ---------------------------------------------------------------------------
 // Episodic inclusive prefix sum, forward, exact in uint32 (two's complement):
 // a = 0 at a row start or after a done step, else 1; b = x.
 // ---------------------------------------------------------------------------
-struct PrefixSumOp {
-  static constexpr int kRegs = 40, kRegsLookback = 32;  // registers per thread, chosen by measurement
+template <int K_ = kTile>
+struct PrefixSumOpT {
+  static constexpr int K = K_;  // steps per thread
+  static constexpr int kRegs = 56, kRegsLookback = 56;  // registers per thread, chosen by measurement
   using V = uint32_t;
   static constexpr bool kBackward = false;
   struct Args {
@@ -483,32 +533,33 @@ struct PrefixSumOp {
     int32_t *out;
   };
   struct Raw {
-    uint32_t x[8];
+    uint32_t x[K];
     uint32_t done;
     uint32_t halo;
   };
   static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &, int lane, uint32_t,
                                               Flags f, Raw &w) {
-    ld8(p.x, tl, w.x);
+    ld_tile(p.x, tl, w.x);
     w.done = f.term | f.trunc;
     w.halo = 0u;
     if (lane == 0 && tl.i0 > 0u && tl.nvalid > 0)
       w.halo = ((p.term && __ldg(p.term + tl.i0 - 1u)) || (p.trunc && __ldg(p.trunc + tl.i0 - 1u))) ? 1u : 0u;
   }
   static __device__ __forceinline__ void fetch_boundary(const Args &, const Tile &, const FastDiv &, Raw &) {}
-  static __device__ __forceinline__ uint32_t nbr_of(const Raw &w) { return (w.done >> 7) & 1u; }
+  static __device__ __forceinline__ uint32_t nbr_of(const Raw &w) { return (w.done >> (K - 1)) & 1u; }
   static __device__ __forceinline__ uint32_t halo_of(const Raw &w) { return w.halo; }
   static __device__ __forceinline__ void coef(const Args &, const Tile &tl, const FastDiv &, Raw &w, uint32_t prev7,
-                                              Aff<uint32_t> (&c)[8]) {
-    const uint32_t cut = (((w.done << 1) | prev7) | tl.edge) & 0xffu;
+                                              Aff<uint32_t> (&c)[K]) {
+    const uint32_t cut = (((w.done << 1) | prev7) | tl.edge) & ((1u << K) - 1u);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) c[k] = Aff<uint32_t>{((cut >> k) & 1u) ^ 1u, w.x[k]};
+    for (int k = 0; k < K; ++k) c[k] = Aff<uint32_t>{((cut >> k) & 1u) ^ 1u, w.x[k]};
   }
-  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<uint32_t> (&)[8],
-                                              const uint32_t (&x)[8], const uint32_t (&)[8]) {
-    st8(p.out, tl, x);
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<uint32_t> (&)[K],
+                                              const uint32_t (&x)[K], const uint32_t (&)[K]) {
+    st_tile(p.out, tl, x);
   }
 };
+using PrefixSumOp = PrefixSumOpT<16>;  // 16 steps per thread: measured faster
 
 // ---------------------------------------------------------------------------
 // Generic affine scan: the pages' unified recurrence with its coefficients
@@ -519,8 +570,9 @@ struct PrefixSumOp {
 // b + a init (init NULL: 0).  The reset flags travel in the flag slot of
 // `term`; `trunc` is NULL.
 // ---------------------------------------------------------------------------
-template <bool BWD, class E = float>
+template <bool BWD, class E = float, int K_ = kTile>
 struct AffineOp {
+  static constexpr int K = K_;  // steps per thread
   static constexpr int kRegs = 40, kRegsLookback = 40;  // registers per thread, chosen by measurement
   using V = float;
   static constexpr bool kBackward = BWD;
@@ -530,14 +582,14 @@ struct AffineOp {
     E *out;
   };
   struct Raw {
-    float a[8], b[8];
+    float a[K], b[K];
     Flags f;
     float ev;  // init of the tile's row edge
   };
   static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int, uint32_t,
                                               Flags f, Raw &w) {
-    ld8(p.a, tl, w.a);
-    ld8(p.b, tl, w.b);
+    ld_tile(p.a, tl, w.a);
+    ld_tile(p.b, tl, w.b);
     w.f = f;
     w.ev = edge_value(p.init, tl, fd);
   }
@@ -545,20 +597,20 @@ struct AffineOp {
   static __device__ __forceinline__ float nbr_of(const Raw &) { return 0.0f; }
   static __device__ __forceinline__ float halo_of(const Raw &) { return 0.0f; }
   static __device__ __forceinline__ void coef(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w, float,
-                                              Aff<float> (&c)[8]) {
+                                              Aff<float> (&c)[K]) {
     const uint32_t cut = w.f.term | tl.edge;
     const uint32_t init_at = tl.edge & ~w.f.term;  // edge steps that take the initial carry
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < K; ++k) {
       float b = w.b[k];
       if (((init_at >> k) & 1u) && p.init)
         b = fmaf(w.a[k], tl.few_rows ? w.ev : ld1(p.init + tl.n0 + fd.div(tl.t0 + k)), b);
       c[k] = Aff<float>{((cut >> k) & 1u) ? 0.0f : w.a[k], b};
     }
   }
-  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[8],
-                                              const float (&x)[8], const float (&)[8]) {
-    st8(p.out, tl, x);
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &, const Aff<float> (&)[K],
+                                              const float (&x)[K], const float (&)[K]) {
+    st_tile(p.out, tl, x);
   }
 };
 
@@ -571,8 +623,9 @@ struct AffineOp {
 // db = g, da_t = g_t x_prv (0 where reset; x_prv = init[n] at the forward
 // scan's first step), dinit[n] = a g at that first step (0 if it resets).
 // ---------------------------------------------------------------------------
-template <bool R>
+template <bool R, int K_ = kTile>
 struct AffineGradOp {
+  static constexpr int K = K_;  // steps per thread
   static constexpr int kRegs = 56, kRegsLookback = 56;  // registers per thread: no spills
   using V = float;
   static constexpr bool kBackward = !R;  // the adjoint runs against the forward scan
@@ -583,7 +636,7 @@ struct AffineGradOp {
     uint32_t T;
   };
   struct Raw {
-    float a[8], x[8], dy[8];
+    float a[K], x[K], dy[K];
     Flags f;
     float ahalo;  // effective a (0 where reset) of the dependency neighbour past the tile
     float xhalo;  // x of the neighbour past the tile on the other side
@@ -596,15 +649,15 @@ struct AffineGradOp {
     if (tl.few_rows) {
       if (R) {
         const uint32_t rend = T - 1u - tl.t0;
-        e = rend < 8u ? (1u << rend) : 0u;
+        e = rend < uint32_t(K) ? (1u << rend) : 0u;
       } else {
         const uint32_t s = tl.t0 == 0u ? 0u : T - tl.t0;
-        e = s < 8u ? (1u << s) : 0u;
+        e = s < uint32_t(K) ? (1u << s) : 0u;
       }
     } else {
       uint32_t tt = tl.t0;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < K; ++k) {
         if (R ? (tt == T - 1u) : (tt == 0u)) e |= 1u << k;
         if (++tt == T) tt = 0;
       }
@@ -613,21 +666,21 @@ struct AffineGradOp {
   }
   static __device__ __forceinline__ void load(const Args &p, const Tile &tl, const FastDiv &fd, int lane,
                                               uint32_t total, Flags f, Raw &w) {
-    ld8(p.a, tl, w.a);
-    ld8(p.x, tl, w.x);
-    ld8(p.dy, tl, w.dy);
+    ld_tile(p.a, tl, w.a);
+    ld_tile(p.x, tl, w.x);
+    ld_tile(p.dy, tl, w.dy);
     w.f = f;
     w.lane = uint32_t(lane);
     // dependency neighbour past the tile: t+1 (adjoint backward) / t-1 (forward)
     w.ahalo = 0.0f;
-    if (!R && lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total)
-      w.ahalo = (p.term && __ldg(p.term + tl.i0 + 8u)) ? 0.0f : __ldg(p.a + tl.i0 + 8u);
+    if (!R && lane == 31 && tl.nvalid == K && tl.i0 + uint32_t(K) < total)
+      w.ahalo = (p.term && __ldg(p.term + tl.i0 + uint32_t(K))) ? 0.0f : __ldg(p.a + tl.i0 + uint32_t(K));
     if (R && lane == 0 && tl.i0 > 0u && tl.nvalid > 0)
       w.ahalo = (p.term && __ldg(p.term + tl.i0 - 1u)) ? 0.0f : __ldg(p.a + tl.i0 - 1u);
     // the other neighbour, for x_prv: t-1 (R false) / t+1 (R true)
     w.xhalo = 0.0f;
     if (!R && lane == 0 && tl.i0 > 0u && tl.nvalid > 0) w.xhalo = __ldg(p.x + tl.i0 - 1u);
-    if (R && lane == 31 && tl.nvalid == 8 && tl.i0 + 8u < total) w.xhalo = __ldg(p.x + tl.i0 + 8u);
+    if (R && lane == 31 && tl.nvalid == K && tl.i0 + uint32_t(K) < total) w.xhalo = __ldg(p.x + tl.i0 + uint32_t(K));
     w.iv = 0.0f;
     const uint32_t fs = first_steps(tl, p.T);
     if (p.init && tl.few_rows && fs) w.iv = __ldg(p.init + tl.n0 + fd.div(tl.t0 + uint32_t(__ffs(fs) - 1)));
@@ -635,41 +688,41 @@ struct AffineGradOp {
   static __device__ __forceinline__ void fetch_boundary(const Args &, const Tile &, const FastDiv &, Raw &) {}
   // a' of the tile's first step in dependency order comes from the neighbour
   static __device__ __forceinline__ float nbr_of(const Raw &w) {
-    return R ? (((w.f.term >> 7) & 1u) ? 0.0f : w.a[7]) : ((w.f.term & 1u) ? 0.0f : w.a[0]);
+    return R ? (((w.f.term >> (K - 1)) & 1u) ? 0.0f : w.a[K - 1]) : ((w.f.term & 1u) ? 0.0f : w.a[0]);
   }
   static __device__ __forceinline__ float halo_of(const Raw &w) { return w.ahalo; }
   static __device__ __forceinline__ void coef(const Args &, const Tile &tl, const FastDiv &, Raw &w, float nb,
-                                              Aff<float> (&c)[8]) {
+                                              Aff<float> (&c)[K]) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < K; ++k) {
       float an;  // effective a of the following step in forward order
       if (R)
         an = k > 0 ? (((w.f.term >> (k - 1)) & 1u) ? 0.0f : w.a[k > 0 ? k - 1 : 0]) : nb;
       else
-        an = k < 7 ? (((w.f.term >> (k + 1)) & 1u) ? 0.0f : w.a[k < 7 ? k + 1 : 7]) : nb;
+        an = k < K - 1 ? (((w.f.term >> (k + 1)) & 1u) ? 0.0f : w.a[k < K - 1 ? k + 1 : K - 1]) : nb;
       c[k] = Aff<float>{((tl.edge >> k) & 1u) ? 0.0f : an, w.dy[k]};
     }
   }
-  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &w, const Aff<float> (&)[8],
-                                              const float (&g)[8], const float (&)[8]) {
-    st8(p.db, tl, g);
+  static __device__ __forceinline__ void emit(const Args &p, const Tile &tl, const Raw &w, const Aff<float> (&)[K],
+                                              const float (&g)[K], const float (&)[K]) {
+    st_tile(p.db, tl, g);
     if (!p.da && !p.dinit) return;
     // x_prv of each step: the other neighbour, by shuffle across the lane edge
-    const float mine = R ? w.x[0] : w.x[7];
+    const float mine = R ? w.x[0] : w.x[K - 1];
     float other = R ? __shfl_down_sync(0xffffffffu, mine, 1) : __shfl_up_sync(0xffffffffu, mine, 1);
     if (R ? w.lane == 31u : w.lane == 0u) other = w.xhalo;
     const uint32_t fs = first_steps(tl, p.T);
-    float da[8];
+    float da[K];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      float xp = R ? (k < 7 ? w.x[k < 7 ? k + 1 : 7] : other) : (k > 0 ? w.x[k > 0 ? k - 1 : 0] : other);
+    for (int k = 0; k < K; ++k) {
+      float xp = R ? (k < K - 1 ? w.x[k < K - 1 ? k + 1 : K - 1] : other) : (k > 0 ? w.x[k > 0 ? k - 1 : 0] : other);
       if ((fs >> k) & 1u)
         xp = !p.init ? 0.0f : (tl.few_rows ? w.iv : __ldg(p.init + tl.n0 + (tl.t0 + k) / p.T));
       da[k] = ((w.f.term >> k) & 1u) ? 0.0f : g[k] * xp;
       if (p.dinit && ((fs >> k) & 1u))
         p.dinit[tl.n0 + (tl.t0 + k) / p.T] = ((w.f.term >> k) & 1u) ? 0.0f : w.a[k] * g[k];
     }
-    if (p.da) st8(p.da, tl, da);
+    if (p.da) st_tile(p.da, tl, da);
   }
 };
 

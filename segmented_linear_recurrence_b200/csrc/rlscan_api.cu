@@ -232,11 +232,27 @@ bool valid_block(int64_t b) { return b >= 128 && b <= 512 && b % 64 == 0; }
 // first step (0 if one row does not fit).  k rows span k T steps, whose tiles
 // number k T / tile when k T is a multiple of the tile (every block then
 // starts aligned) and at most (k T + 2 tile - 2) / tile otherwise.
-int64_t rows_per_block(int64_t T, int block, int64_t tile = kTile) {
+int64_t rows_per_block(int64_t T, int block, int64_t tile) {
   auto tiles = [T, tile](int64_t k) { return (k * T) % tile == 0 ? k * T / tile : (k * T + 2 * tile - 2) / tile; };
   int64_t k = tile * block / T;
   while (k > 0 && tiles(k) > block) --k;
   return k;
+}
+
+// Steps per thread of each estimator's kernel (Op::K).
+int tile_steps(rlscan_estimator est) {
+  switch (est) {
+    case RLSCAN_EST_GAE: return GaeOp::K;
+    case RLSCAN_EST_VTRACE: return VtraceOp::K;
+    case RLSCAN_EST_TD_LAMBDA: return TdLambdaOp::K;
+    case RLSCAN_EST_DISCOUNTED_RETURN: return DiscountedOp::K;
+    case RLSCAN_EST_ELIG_TRACE: return EligOp::K;
+    case RLSCAN_EST_EPISODIC_PREFIX_SUM: return PrefixSumOp::K;
+    case RLSCAN_EST_AFFINE_SCAN: return AffineOp<false>::K;
+    case RLSCAN_EST_AFFINE_SCAN_GRAD: return AffineGradOp<false>::K;
+    case RLSCAN_EST_AFFINE_SCAN_BF16: return AffineOp<false, __nv_bfloat16>::K;
+    default: return 4;  // Retrace: its own 4-step tiles
+  }
 }
 
 Plan make_plan(rlscan_estimator est, int64_t N, int64_t T, int64_t A) {
@@ -271,13 +287,14 @@ Plan make_plan(rlscan_estimator est, int64_t N, int64_t T, int64_t A) {
   } else {
     // Rows plan where a row fits a block: the block size whose threads the
     // rows fill best (the smaller one on a tie); else the look-back plan.
+    const int K = tile_steps(est);
     int64_t best_k = 0;
     pl.block = 256;
     double best_fill = 0.0;
     for (int b : kBlocks) {
       if (valid_block(fb) && b != fb) continue;
-      const int64_t k = rows_per_block(T, b);
-      const double fill = double(k * T) / double(int64_t(kTile) * b);
+      const int64_t k = rows_per_block(T, b, K);
+      const double fill = double(k * T) / double(int64_t(K) * b);
       if (k > 0 && fill > best_fill + 1e-9) {
         best_fill = fill;
         best_k = k;
@@ -287,7 +304,7 @@ Plan make_plan(rlscan_estimator est, int64_t N, int64_t T, int64_t A) {
     if (valid_block(fb)) pl.block = int(fb);
     pl.lookback = force_lb || best_k == 0;
     if (pl.lookback) {
-      pl.L = uint32_t(kTile) * uint32_t(pl.block);
+      pl.L = uint32_t(K) * uint32_t(pl.block);
     } else {
       pl.rows_per_block = best_k;
       pl.L = uint32_t(best_k * T);

@@ -6,19 +6,19 @@
 // on chip, runs the associative scan on chip and writes each output once, so
 // a call moves each element through HBM exactly once.
 //
-// Work decomposition (ours, B200-first).  Thread j of a block owns the 8
-// consecutive steps starting at base + 8j, base a multiple of 8 (one 256-bit
-// load per fp32 array).  Two plans:
+// Work decomposition (ours, B200-first).  Thread j of a block owns the K
+// (= Op::K, 8 or 16) consecutive steps starting at base + K j, base a
+// multiple of K (one 256-bit load per 8 steps of an fp32 array).  Two plans:
 //   LB == false (rows fit a block): block b owns rows [b k, (b + 1) k), i.e.
 //     the steps [b span, (b + 1) span) with span = k T.  Its tiles start at
-//     that range's first step rounded down to a multiple of 8, so the first
+//     that range's first step rounded down to a multiple of K, so the first
 //     and last tile may hold steps of the neighbouring blocks: those are
 //     loaded (in bounds, harmless) but neither scanned nor stored.  Every
 //     block's range starts and ends on row edges, so no block needs a carry
 //     from another.  The host picks k (and the block size) to fill the
 //     block's threads.
 //   LB == true (rows longer than a block): the launch's steps are one flat
-//     sequence cut into chunks of L = 8 * BLOCK steps; chunks take tickets
+//     sequence cut into chunks of L = K * BLOCK steps; chunks take tickets
 //     in dependency order and hand carries over with a decoupled look-back
 //     (scan_core.cuh).  Because the coefficient builders put a = 0 on each
 //     row's dependency edge, chunks may straddle rows freely: the flat scan
@@ -52,20 +52,20 @@ struct ScanGeom {
   LookbackCtl lb;         // ticket / done / epoch counters and descriptors (look-back only)
 };
 
-// Steps, row position and row edges of the tile at step i0 (a multiple of 8)
+// Steps, row position and row edges of the K-step tile at step i0 (a multiple of K)
 // of a block that owns the steps [lo, hi), i0 + 8 > lo.
-template <bool BWD>
+template <bool BWD, int K>
 __device__ __forceinline__ Tile make_tile(const ScanGeom &g, const FastDiv &fd, uint32_t i0, uint32_t lo,
                                           uint32_t hi) {
   Tile t;
   t.i0 = i0;
-  t.nvalid = i0 < g.total ? int(min(uint32_t(kTile), g.total - i0)) : 0;
-  uint32_t v = i0 < hi ? (1u << min(uint32_t(kTile), hi - i0)) - 1u : 0u;
+  t.nvalid = i0 < g.total ? int(min(uint32_t(K), g.total - i0)) : 0;
+  uint32_t v = i0 < hi ? (1u << min(uint32_t(K), hi - i0)) - 1u : 0u;
   if (i0 < lo) v &= ~((1u << (lo - i0)) - 1u);
   t.valid = v;
-  t.fast = g.vec != 0u && t.nvalid == kTile;
-  t.full = t.fast && v == 0xffu;
-  t.few_rows = g.T >= uint32_t(kTile);
+  t.fast = g.vec != 0u && t.nvalid == K;
+  t.full = t.fast && v == (K == 32 ? 0xffffffffu : (1u << K) - 1u);
+  t.few_rows = g.T >= uint32_t(K);
   t.n0 = 0;
   t.t0 = 0;
   t.edge = 0;
@@ -76,15 +76,15 @@ __device__ __forceinline__ Tile make_tile(const ScanGeom &g, const FastDiv &fd, 
   if (t.few_rows) {
     if (BWD) {
       const uint32_t rend = g.T - 1u - t.t0;
-      e = rend < uint32_t(kTile) ? (1u << rend) : 0u;
+      e = rend < uint32_t(K) ? (1u << rend) : 0u;
     } else {
       const uint32_t s = t.t0 == 0u ? 0u : g.T - t.t0;
-      e = s < uint32_t(kTile) ? (1u << s) : 0u;
+      e = s < uint32_t(K) ? (1u << s) : 0u;
     }
   } else {
     uint32_t tt = t.t0;
 #pragma unroll
-    for (int k = 0; k < kTile; ++k) {
+    for (int k = 0; k < K; ++k) {
       if (BWD ? (tt == g.T - 1u) : (tt == 0u)) e |= 1u << k;
       if (++tt == g.T) tt = 0;
     }
@@ -137,10 +137,21 @@ constexpr int min_blocks_per_sm() {
 // with cp.async and reads them back itself (no barrier needed).
 // 16-byte aligned: the 8-byte cp.async copies need an 8-byte aligned
 // destination, whatever the shared-memory layout around the slots.
+template <int K>
 struct __align__(16) FlagSlot {
-  uint32_t term[2], trunc[2];
+  uint32_t term[K / 4], trunc[K / 4];
 };
-static_assert(alignof(FlagSlot) >= 8 && sizeof(FlagSlot) == 16, "cp.async destinations must stay aligned");
+static_assert(alignof(FlagSlot<8>) >= 8 && sizeof(FlagSlot<8>) == 16, "cp.async destinations must stay aligned");
+static_assert(alignof(FlagSlot<16>) >= 8 && sizeof(FlagSlot<16>) == 32, "cp.async destinations must stay aligned");
+
+// Flag masks from a prefetched slot (bit k: step k).
+template <int K>
+__device__ __forceinline__ uint32_t slot_mask(const uint32_t (&w)[K / 4]) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < K / 4; ++j) m |= nonzero_bytes4(w[j]) << (4 * j);
+  return m;
+}
 
 __device__ __forceinline__ void cp_async8(void *dst_smem, const void *src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst_smem))),
@@ -153,7 +164,7 @@ template <class Op, int BLOCK, bool LB>
 struct ScanSmem {
   using V = typename Op::V;
   static constexpr int W = BLOCK / 32;
-  static constexpr int kParked = LB ? int(sizeof(Aff<V>) * kTile / 4) : 1;
+  static constexpr int kParked = LB ? int(sizeof(Aff<V>) * Op::K / 4) : 1;
   Aff<V> wagg[W];
   Aff<V> wagg2[2][W];  // rows plan: double-buffered by chunk
   V wcarry[W];
@@ -168,19 +179,20 @@ struct ScanSmem {
 template <class Op>
 __device__ __forceinline__ void resweep_and_emit(const typename Op::Args &p, const Tile &tl,
                                                  const typename Op::Raw &w,
-                                                 const Aff<typename Op::V> (&c)[kTile], typename Op::V x) {
+                                                 const Aff<typename Op::V> (&c)[Op::K], typename Op::V x) {
   using V = typename Op::V;
-  V xs[kTile], xd[kTile];
+  constexpr int K = Op::K;
+  V xs[K], xd[K];
   if (Op::kBackward) {
 #pragma unroll
-    for (int k = kTile - 1; k >= 0; --k) {
+    for (int k = K - 1; k >= 0; --k) {
       xd[k] = x;
       x = apply(c[k], x);
       xs[k] = x;
     }
   } else {
 #pragma unroll
-    for (int k = 0; k < kTile; ++k) {
+    for (int k = 0; k < K; ++k) {
       xd[k] = x;
       x = apply(c[k], x);
       xs[k] = x;
@@ -202,7 +214,8 @@ __device__ __forceinline__ void scan_chunk(const typename Op::Args &p, const Sca
   using Raw = typename Op::Raw;
   constexpr bool BWD = Op::kBackward;
   constexpr int W = BLOCK / 32;
-  constexpr uint32_t L = uint32_t(kTile) * BLOCK;
+  constexpr int K = Op::K;
+  constexpr uint32_t L = uint32_t(K) * BLOCK;
   const int lane = tid & 31, warp = tid >> 5;
 
   // a1: every load of the tile goes out together.
@@ -219,24 +232,24 @@ __device__ __forceinline__ void scan_chunk(const typename Op::Args &p, const Sca
   if constexpr (!early) Op::fetch_boundary(p, tl, fd, w);
 
   // a2: coefficients in registers.
-  Aff<V> c[kTile];
+  Aff<V> c[K];
   Op::coef(p, tl, fd, w, from, c);
-  if (tl.valid != 0xffu) {
+  if (tl.valid != (K == 32 ? 0xffffffffu : (1u << K) - 1u)) {
 #pragma unroll
-    for (int k = 0; k < kTile; ++k)
+    for (int k = 0; k < K; ++k)
       if (!((tl.valid >> k) & 1u)) c[k] = aff_identity<V>();
   }
 
-  // a4: sequential composite of the thread's 8 steps, in dependency order.
+  // a4: sequential composite of the thread's K steps, in dependency order.
   Aff<V> agg;
   if (BWD) {
-    agg = c[kTile - 1];
+    agg = c[K - 1];
 #pragma unroll
-    for (int k = kTile - 2; k >= 0; --k) agg = compose(c[k], agg);
+    for (int k = K - 2; k >= 0; --k) agg = compose(c[k], agg);
   } else {
     agg = c[0];
 #pragma unroll
-    for (int k = 1; k < kTile; ++k) agg = compose(c[k], agg);
+    for (int k = 1; k < K; ++k) agg = compose(c[k], agg);
   }
 
   // a5: warp scan.
@@ -295,7 +308,8 @@ template <class Op, int BLOCK, bool LB>
 __global__ void __launch_bounds__(BLOCK, (min_blocks_per_sm<Op, BLOCK, LB>()))
     scan_kernel(const typename Op::Args p, const ScanGeom g) {
   constexpr bool BWD = Op::kBackward;
-  constexpr uint32_t L = uint32_t(kTile) * BLOCK;
+  constexpr int K = Op::K;
+  constexpr uint32_t L = uint32_t(K) * BLOCK;
   static_assert(BLOCK % 32 == 0 && BLOCK / 32 <= 32, "block must be whole warps, at most 32");
 
   __shared__ ScanSmem<Op, BLOCK, LB> sm;
@@ -315,39 +329,42 @@ __global__ void __launch_bounds__(BLOCK, (min_blocks_per_sm<Op, BLOCK, LB>()))
     if (ticket >= g.nchunks) return;  // counter left inconsistent by an aborted launch
     const uint32_t chunk = BWD ? g.nchunks - 1u - ticket : ticket;
     const uint32_t lo = chunk * L, hi = min(lo + L, g.total);
-    const Tile tl = make_tile<BWD>(g, fd, lo + uint32_t(kTile) * uint32_t(tid), lo, hi);
-    const Flags f{ld8_flags(p.term, tl), ld8_flags(p.trunc, tl)};
+    const Tile tl = make_tile<BWD, K>(g, fd, lo + uint32_t(K) * uint32_t(tid), lo, hi);
+    const Flags f{ld_flags<K>(p.term, tl), ld_flags<K>(p.trunc, tl)};
     scan_chunk<Op, BLOCK, LB>(p, g, fd, sm, chunk, tl, f, tid, 0);
   } else {
     // Rows plan, persistent: the block takes chunks blockIdx.x, + gridDim.x,
     // ...  While it scans one chunk, its threads prefetch the next chunk's
     // flag bytes, so the trunc_value loads that depend on them go out with
     // the chunk's other loads instead of a memory round trip later.
-    __shared__ FlagSlot slots[2][BLOCK];
+    __shared__ FlagSlot<K> slots[2][BLOCK];
     auto tile_of = [&](uint32_t chunk) {
       const uint32_t lo = chunk * g.span, hi = min(lo + g.span, g.total);
-      return make_tile<BWD>(g, fd, (lo & ~uint32_t(kTile - 1)) + uint32_t(kTile) * uint32_t(tid), lo, hi);
+      return make_tile<BWD, K>(g, fd, (lo & ~uint32_t(K - 1)) + uint32_t(K) * uint32_t(tid), lo, hi);
     };
     // Prefetch needs the 8-byte copies in bounds and aligned: full tiles of
     // vectorised launches only; any other tile loads its flags directly.
     // Only the next tile's first step is computed ahead; its full geometry
     // is built after the current chunk, to keep the loop light in registers.
-    auto prefetch = [&](uint32_t chunk, FlagSlot &slot) {
-      const uint32_t i0 = ((chunk * g.span) & ~uint32_t(kTile - 1)) + uint32_t(kTile) * uint32_t(tid);
-      if (g.vec == 0u || i0 + uint32_t(kTile) > g.total) return false;
-      if (p.term) cp_async8(slot.term, p.term + i0);
-      if (p.trunc) cp_async8(slot.trunc, p.trunc + i0);
+    auto prefetch = [&](uint32_t chunk, FlagSlot<K> &slot) {
+      const uint32_t i0 = ((chunk * g.span) & ~uint32_t(K - 1)) + uint32_t(K) * uint32_t(tid);
+      if (g.vec == 0u || i0 + uint32_t(K) > g.total) return false;
+#pragma unroll
+      for (int j = 0; j < K / 8; ++j) {
+        if (p.term) cp_async8(slot.term + 2 * j, p.term + i0 + 8 * j);
+        if (p.trunc) cp_async8(slot.trunc + 2 * j, p.trunc + i0 + 8 * j);
+      }
       asm volatile("cp.async.commit_group;" ::: "memory");
       return true;
     };
-    // When every chunk starts on an 8-step boundary (k T a multiple of 8), a
+    // When every chunk starts on a K-step boundary (k T a multiple of K), a
     // thread's tile has the same offset, time and row edges in every full
     // chunk: only its first step and row move.  Holding that tile across the
     // loop costs registers, so estimators on a 32-register budget (where it
     // measured slower) rebuild the tile per chunk instead.
     constexpr bool kKeepTile = Op::kRegs >= 40;
-    const bool aligned = kKeepTile && (g.span % uint32_t(kTile)) == 0u && g.span <= g.total;
-    Tile inv = make_tile<BWD>(g, fd, uint32_t(kTile) * uint32_t(tid), 0u, g.span);
+    const bool aligned = kKeepTile && (g.span % uint32_t(K)) == 0u && g.span <= g.total;
+    Tile inv = make_tile<BWD, K>(g, fd, uint32_t(K) * uint32_t(tid), 0u, g.span);
     if (inv.valid == 0u) {  // thread beyond the chunk's steps: loads nothing
       inv.nvalid = 0;
       inv.fast = inv.full = false;
@@ -359,7 +376,7 @@ __global__ void __launch_bounds__(BLOCK, (min_blocks_per_sm<Op, BLOCK, LB>()))
       Tile tl;
       if (aligned && lo + g.span <= g.total) {
         tl = inv;
-        tl.i0 = lo + uint32_t(kTile) * uint32_t(tid);
+        tl.i0 = lo + uint32_t(K) * uint32_t(tid);
         tl.n0 = inv.n0 + chunk * g.rows_per_chunk;
       } else {
         tl = tile_of(chunk);
@@ -367,11 +384,11 @@ __global__ void __launch_bounds__(BLOCK, (min_blocks_per_sm<Op, BLOCK, LB>()))
       Flags f;
       if (have) {
         asm volatile("cp.async.wait_group 0;" ::: "memory");
-        const FlagSlot &s = slots[buf][tid];
-        f.term = p.term ? nonzero_bytes4(s.term[0]) | (nonzero_bytes4(s.term[1]) << 4) : 0u;
-        f.trunc = p.trunc ? nonzero_bytes4(s.trunc[0]) | (nonzero_bytes4(s.trunc[1]) << 4) : 0u;
+        const FlagSlot<K> &s = slots[buf][tid];
+        f.term = p.term ? slot_mask<K>(s.term) : 0u;
+        f.trunc = p.trunc ? slot_mask<K>(s.trunc) : 0u;
       } else {
-        f = Flags{ld8_flags(p.term, tl), ld8_flags(p.trunc, tl)};
+        f = Flags{ld_flags<K>(p.term, tl), ld_flags<K>(p.trunc, tl)};
       }
       const uint32_t next = chunk + gridDim.x;
       have = next < g.nchunks && prefetch(next, slots[buf ^ 1][tid]);

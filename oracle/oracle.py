@@ -35,6 +35,7 @@ def bind(lib):
         "rlo_episodic_prefix_sum": [i64, i64, vp, vp, vp, vp, vp],
         "rlo_affine_scan": [i64, i64, vp, vp, vp, vp, ctypes.c_int, vp],
         "rlo_affine_scan_grad": [i64, i64, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp],
+        "rlo_affine_scan_tm": [i64, i64, vp, vp, vp, vp, ctypes.c_int, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -174,6 +175,20 @@ def affine_scan(a, b, reset=None, init=None, reverse=False):
     return out
 
 
+def affine_scan_tm(a, b, reset=None, init=None, reverse=False):
+    """affine_scan on time-major [T, N] arrays (init [N]); returns [T, N]."""
+    a = np.asarray(a)
+    if a.ndim != 2:
+        raise ValueError("time-major arrays must be 2-D [T, N]")
+    T, N = int(a.shape[0]), int(a.shape[1])
+    keep = [_p(a, np.float32), _p(b, np.float32), _p(reset, np.uint8), _p(init, np.float32)]
+    out = np.empty((T, N), np.float64)
+    rc = _load().rlo_affine_scan_tm(N, T, *[k[1] for k in keep], 1 if reverse else 0,
+                                    out.ctypes.data_as(ctypes.c_void_p))
+    _check(rc, "affine_scan_tm")
+    return out
+
+
 def affine_scan_grad(a, x, dy, reset=None, init=None, reverse=False):
     """Adjoint of affine_scan: returns (da, db, dinit) for upstream dy, given
     the forward output x (all fp64)."""
@@ -203,4 +218,4 @@ def run(name, inp, **scal):
 
 
 __all__ = ["gae", "td_lambda", "discounted_return", "vtrace", "retrace", "elig_trace",
-           "episodic_prefix_sum", "affine_scan", "affine_scan_grad", "run"]
+           "episodic_prefix_sum", "affine_scan", "affine_scan_grad", "affine_scan_tm", "run"]

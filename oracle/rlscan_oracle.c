@@ -358,3 +358,24 @@ int rlo_affine_scan_grad(int64_t N, int64_t T, const float *a, const float *x,
   }
   return 0;
 }
+
+/* rlo_affine_scan on time-major arrays: element (t, n) of a, b, reset and x
+ * at t * N + n (each time step a contiguous row of the N environments);
+ * init is [N].  Same recurrence, same scan order per environment. */
+int rlo_affine_scan_tm(int64_t N, int64_t T, const float *a, const float *b,
+                       const uint8_t *reset, const float *init, int reverse,
+                       double *x) {
+  if (bad_dims(N, T)) return -1;
+  for (int64_t n = 0; n < N; ++n) {
+    double carry = init ? (double)init[n] : 0.0;
+    for (int64_t k = 0; k < T; ++k) {
+      const int64_t t = reverse ? T - 1 - k : k;
+      const int64_t i = t * N + n;
+      double v = (double)b[i];
+      if (!(reset && reset[i])) v += (double)a[i] * carry;
+      x[i] = v;
+      carry = v;
+    }
+  }
+  return 0;
+}

@@ -674,3 +674,26 @@ def test_affine_grad_zero_coefficient():
     xp = np.concatenate([d["init"][:, None], x[:, :-1]], axis=1).astype(np.float64)
     np.testing.assert_allclose(da, dy.astype(np.float64) * xp, rtol=1e-15)
     np.testing.assert_array_equal(dinit, np.zeros(2))
+
+
+# --------------------------------------------------------------------------
+# time-major affine scan ([T, N] arrays): pinned against the non-recursive
+# sum on the transposed rows, and against the row-major routine
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_affine_tm_matches_bruteforce_on_transpose(reverse):
+    d = synthetic.make_affine_inputs(5, 9, seed=51, p_reset=0.2, a_low=-1.1, a_high=1.1)
+    tm = lambda v: None if v is None else np.ascontiguousarray(v.T)  # noqa: E731
+    got = oracle.affine_scan_tm(tm(d["a"]), tm(d["b"]), tm(d["reset"]), d["init"], reverse=reverse)
+    want = bf_affine(d["a"], d["b"], d["reset"], d["init"], reverse)
+    np.testing.assert_allclose(got, want.T, rtol=1e-12, atol=1e-12)
+
+
+def test_affine_tm_is_row_major_on_transposed_arrays():
+    d = synthetic.make_affine_inputs(7, 300, seed=52, p_reset=0.05)
+    tm = lambda v: None if v is None else np.ascontiguousarray(v.T)  # noqa: E731
+    for reverse in (False, True):
+        got = oracle.affine_scan_tm(tm(d["a"]), tm(d["b"]), tm(d["reset"]), d["init"], reverse=reverse)
+        want = oracle.affine_scan(d["a"], d["b"], d["reset"], d["init"], reverse=reverse)
+        np.testing.assert_array_equal(got, want.T)

@@ -263,6 +263,48 @@ rlscan_status rlscan_affine_scan_grad(const float *a, const float *x, const floa
                                       int64_t T, int32_t reverse, rlscan_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Time-major layout (the memory-layout option of the rl-triton API page,
+ * Hugging Face model card, "Key Features": contiguous vs strided).  Each call
+ * below takes the same arguments, applies the same checks and computes the
+ * same values as the row-major call of the same name without "_tm", but every
+ * per-step array is time-major [T,N]: element (t, n) at t * N + n, so each time
+ * step is one contiguous run of the N environments (the layout of rollout
+ * buffers filled one vectorised environment step at a time).  Per-environment
+ * arrays (bootstrap, init_trace, init) stay [N].  Retrace and the bf16 and
+ * adjoint scans are row-major only.
+ * - Limits: N <= 2^26 and fewer than 2^31 thread-block chunks (T / 64 times
+ *   N / 32, roughly); larger calls return RLSCAN_ERR_INVALID_ARG.
+ * - Scratch: windows longer than one block's chunk (64 steps) hand carries
+ *   along T through the stream's workspace, 16 bytes per environment per
+ *   chunk (rlscan_query_plan_tm reports it).
+ * - RLSCAN_OPT_FORCE_LOOKBACK applies (shorter chunks, so carries chain even
+ *   for short windows); RLSCAN_OPT_FORCE_BLOCK and _FORCE_SCALAR do not (256
+ *   threads, one scalar access per step and array, any alignment of 4 bytes).
+ * ------------------------------------------------------------------------- */
+rlscan_status rlscan_gae_tm(const float *rewards, const float *values, const float *bootstrap,
+                            const uint8_t *terminated, const uint8_t *truncated, const float *trunc_value,
+                            float *advantages, float *returns, int64_t N, int64_t T, float gamma, float lambda,
+                            rlscan_stream_t stream);
+rlscan_status rlscan_vtrace_tm(const float *log_rhos, const float *rewards, const float *values,
+                               const float *bootstrap, const uint8_t *terminated, const uint8_t *truncated,
+                               const float *trunc_value, float *vs, float *pg_advantages, int64_t N, int64_t T,
+                               float gamma, float lambda, float rho_bar, float c_bar, rlscan_stream_t stream);
+rlscan_status rlscan_td_lambda_tm(const float *rewards, const float *values, const float *bootstrap,
+                                  const uint8_t *terminated, const uint8_t *truncated, const float *trunc_value,
+                                  float *returns, int64_t N, int64_t T, float gamma, float lambda,
+                                  rlscan_stream_t stream);
+rlscan_status rlscan_discounted_return_tm(const float *rewards, const float *bootstrap, const uint8_t *terminated,
+                                          const uint8_t *truncated, const float *trunc_value, float *returns,
+                                          int64_t N, int64_t T, float gamma, rlscan_stream_t stream);
+rlscan_status rlscan_elig_trace_tm(const float *inputs, const float *init_trace, const uint8_t *terminated,
+                                   const uint8_t *truncated, float *traces, int64_t N, int64_t T, float gamma,
+                                   float lambda, rlscan_stream_t stream);
+rlscan_status rlscan_episodic_prefix_sum_tm(const int32_t *x, const uint8_t *terminated, const uint8_t *truncated,
+                                            int32_t *out, int64_t N, int64_t T, rlscan_stream_t stream);
+rlscan_status rlscan_affine_scan_tm(const float *a, const float *b, const uint8_t *reset, const float *init,
+                                    float *x, int64_t N, int64_t T, int32_t reverse, rlscan_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Status, workspace and configuration.
  * ------------------------------------------------------------------------- */
 
@@ -315,6 +357,11 @@ typedef struct rlscan_plan_info {
 
 rlscan_status rlscan_query_plan(rlscan_estimator estimator, int64_t N, int64_t T, int64_t A,
                                 rlscan_plan_info *info);
+/* The same for the time-major calls (estimators with a "_tm" entry point;
+ * others give RLSCAN_ERR_INVALID_ARG).  chunks counts thread blocks, each a
+ * chunk of chunk_steps steps: K steps x up to 8 time slices x 32 environments
+ * per column group. */
+rlscan_status rlscan_query_plan_tm(rlscan_estimator estimator, int64_t N, int64_t T, rlscan_plan_info *info);
 
 /* Process-wide options (all default 0 unless stated). */
 typedef enum rlscan_option {

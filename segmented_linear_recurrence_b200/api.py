@@ -24,7 +24,9 @@ __all__ = [
     "rlscan_discounted_return", "rlscan_elig_trace", "rlscan_episodic_prefix_sum",
     "rlscan_affine_scan", "rlscan_affine_scan_grad", "rlscan_affine_scan_bf16", "rlscan_sync_status", "rlscan_status_string", "rlscan_release_workspaces",
     "rlscan_abi_version", "rlscan_query_plan", "rlscan_set_option", "rlscan_get_option",
-    "rlscan_reserve_workspace",
+    "rlscan_reserve_workspace", "rlscan_gae_tm", "rlscan_vtrace_tm", "rlscan_td_lambda_tm",
+    "rlscan_discounted_return_tm", "rlscan_elig_trace_tm", "rlscan_episodic_prefix_sum_tm",
+    "rlscan_affine_scan_tm", "rlscan_query_plan_tm",
     "STATUS", "OPTIONS", "ESTIMATOR_IDS", "LIB_PATH",
 ]
 
@@ -65,6 +67,14 @@ _SIGNATURES = {
     "rlscan_affine_scan": [_VP] * 5 + [_I64, _I64, ctypes.c_int32, _VP],
     "rlscan_affine_scan_grad": [_VP] * 8 + [_I64, _I64, ctypes.c_int32, _VP],
     "rlscan_affine_scan_bf16": [_VP] * 5 + [_I64, _I64, ctypes.c_int32, _VP],
+    "rlscan_gae_tm": [_VP] * 8 + [_I64, _I64, _F, _F, _VP],
+    "rlscan_vtrace_tm": [_VP] * 9 + [_I64, _I64, _F, _F, _F, _F, _VP],
+    "rlscan_td_lambda_tm": [_VP] * 7 + [_I64, _I64, _F, _F, _VP],
+    "rlscan_discounted_return_tm": [_VP] * 6 + [_I64, _I64, _F, _VP],
+    "rlscan_elig_trace_tm": [_VP] * 5 + [_I64, _I64, _F, _F, _VP],
+    "rlscan_episodic_prefix_sum_tm": [_VP] * 4 + [_I64, _I64, _VP],
+    "rlscan_affine_scan_tm": [_VP] * 5 + [_I64, _I64, ctypes.c_int32, _VP],
+    "rlscan_query_plan_tm": [_I, _I64, _I64, ctypes.POINTER(PlanInfo)],
     "rlscan_sync_status": [_VP],
     "rlscan_release_workspaces": [],
     "rlscan_reserve_workspace": [_I64, _VP],
@@ -176,10 +186,11 @@ class _Call:
         return tuple(res)
 
 
-def _nt(x, name):
+def _nt(x, name, tm=False):
+    """(N, T) of a per-step tensor: [N, T] row-major, or [T, N] time-major."""
     if not isinstance(x, torch.Tensor) or x.dim() != 2:
-        raise ValueError(f"{name}: per-step inputs must be 2-D [N, T] tensors")
-    return int(x.shape[0]), int(x.shape[1])
+        raise ValueError(f"{name}: per-step inputs must be 2-D {'[T, N]' if tm else '[N, T]'} tensors")
+    return (int(x.shape[1]), int(x.shape[0])) if tm else (int(x.shape[0]), int(x.shape[1]))
 
 
 # ---------------------------------------------------------------------------
@@ -187,39 +198,43 @@ def _nt(x, name):
 # ---------------------------------------------------------------------------
 
 def rlscan_gae(rewards, values, bootstrap, terminated=None, truncated=None, trunc_value=None, *,
-               gamma=0.99, lam=0.95, advantages=None, returns=None, want_returns=True, stream=None):
+               gamma=0.99, lam=0.95, advantages=None, returns=None, want_returns=True, stream=None, _tm=False):
     """GAE advantages and returns.  Returns (advantages, returns or None)."""
-    N, T = _nt(rewards, "rlscan_gae")
-    c = _Call("rlscan_gae", rewards)
-    r = c.tensor(rewards, torch.float32, (N, T), "rewards")
-    v = c.tensor(values, torch.float32, (N, T), "values")
+    name = "rlscan_gae_tm" if _tm else "rlscan_gae"
+    N, T = _nt(rewards, name, _tm)
+    S = (T, N) if _tm else (N, T)
+    c = _Call(name, rewards)
+    r = c.tensor(rewards, torch.float32, S, "rewards")
+    v = c.tensor(values, torch.float32, S, "values")
     b = c.tensor(bootstrap, torch.float32, (N,), "bootstrap")
-    te = c.tensor(terminated, torch.uint8, (N, T), "terminated", required=False)
-    tr = c.tensor(truncated, torch.uint8, (N, T), "truncated", required=False)
-    tv = c.tensor(trunc_value, torch.float32, (N, T), "trunc_value", required=tr is not None)
-    adv = c.output(advantages, torch.float32, (N, T), "advantages")
-    ret = c.output(returns, torch.float32, (N, T), "returns") if (want_returns or returns is not None) else None
-    st = lib().rlscan_gae(c.ptr(r), c.ptr(v), c.ptr(b), c.ptr(te), c.ptr(tr), c.ptr(tv), c.ptr(adv),
+    te = c.tensor(terminated, torch.uint8, S, "terminated", required=False)
+    tr = c.tensor(truncated, torch.uint8, S, "truncated", required=False)
+    tv = c.tensor(trunc_value, torch.float32, S, "trunc_value", required=tr is not None)
+    adv = c.output(advantages, torch.float32, S, "advantages")
+    ret = c.output(returns, torch.float32, S, "returns") if (want_returns or returns is not None) else None
+    st = getattr(lib(), name)(c.ptr(r), c.ptr(v), c.ptr(b), c.ptr(te), c.ptr(tr), c.ptr(tv), c.ptr(adv),
                           c.ptr(ret), N, T, float(gamma), float(lam), c.stream(stream))
     return c.finish(st, (adv, ret))
 
 
 def rlscan_vtrace(log_rhos, rewards, values, bootstrap, terminated=None, truncated=None,
                   trunc_value=None, *, gamma=0.99, lam=1.0, rho_bar=1.0, c_bar=1.0, vs=None,
-                  pg_advantages=None, want_pg=True, stream=None):
+                  pg_advantages=None, want_pg=True, stream=None, _tm=False):
     """V-trace targets vs and policy-gradient advantages.  Returns (vs, pg or None)."""
-    N, T = _nt(rewards, "rlscan_vtrace")
-    c = _Call("rlscan_vtrace", rewards)
-    lr = c.tensor(log_rhos, torch.float32, (N, T), "log_rhos")
-    r = c.tensor(rewards, torch.float32, (N, T), "rewards")
-    v = c.tensor(values, torch.float32, (N, T), "values")
+    name = "rlscan_vtrace_tm" if _tm else "rlscan_vtrace"
+    N, T = _nt(rewards, name, _tm)
+    S = (T, N) if _tm else (N, T)
+    c = _Call(name, rewards)
+    lr = c.tensor(log_rhos, torch.float32, S, "log_rhos")
+    r = c.tensor(rewards, torch.float32, S, "rewards")
+    v = c.tensor(values, torch.float32, S, "values")
     b = c.tensor(bootstrap, torch.float32, (N,), "bootstrap")
-    te = c.tensor(terminated, torch.uint8, (N, T), "terminated", required=False)
-    tr = c.tensor(truncated, torch.uint8, (N, T), "truncated", required=False)
-    tv = c.tensor(trunc_value, torch.float32, (N, T), "trunc_value", required=tr is not None)
-    out_vs = c.output(vs, torch.float32, (N, T), "vs")
-    pg = c.output(pg_advantages, torch.float32, (N, T), "pg_advantages") if (want_pg or pg_advantages is not None) else None
-    st = lib().rlscan_vtrace(c.ptr(lr), c.ptr(r), c.ptr(v), c.ptr(b), c.ptr(te), c.ptr(tr), c.ptr(tv),
+    te = c.tensor(terminated, torch.uint8, S, "terminated", required=False)
+    tr = c.tensor(truncated, torch.uint8, S, "truncated", required=False)
+    tv = c.tensor(trunc_value, torch.float32, S, "trunc_value", required=tr is not None)
+    out_vs = c.output(vs, torch.float32, S, "vs")
+    pg = c.output(pg_advantages, torch.float32, S, "pg_advantages") if (want_pg or pg_advantages is not None) else None
+    st = getattr(lib(), name)(c.ptr(lr), c.ptr(r), c.ptr(v), c.ptr(b), c.ptr(te), c.ptr(tr), c.ptr(tv),
                              c.ptr(out_vs), c.ptr(pg), N, T, float(gamma), float(lam),
                              float(rho_bar), float(c_bar), c.stream(stream))
     return c.finish(st, (out_vs, pg))
@@ -249,78 +264,88 @@ def rlscan_retrace(q, pi, mu_a, actions, rewards, bootstrap, terminated=None, tr
 
 
 def rlscan_td_lambda(rewards, values, bootstrap, terminated=None, truncated=None, trunc_value=None,
-                     *, gamma=0.99, lam=0.95, returns=None, stream=None):
+                     *, gamma=0.99, lam=0.95, returns=None, stream=None, _tm=False):
     """TD(lambda) returns.  Returns the [N, T] returns."""
-    N, T = _nt(rewards, "rlscan_td_lambda")
-    c = _Call("rlscan_td_lambda", rewards)
-    r = c.tensor(rewards, torch.float32, (N, T), "rewards")
-    v = c.tensor(values, torch.float32, (N, T), "values")
+    name = "rlscan_td_lambda_tm" if _tm else "rlscan_td_lambda"
+    N, T = _nt(rewards, name, _tm)
+    S = (T, N) if _tm else (N, T)
+    c = _Call(name, rewards)
+    r = c.tensor(rewards, torch.float32, S, "rewards")
+    v = c.tensor(values, torch.float32, S, "values")
     b = c.tensor(bootstrap, torch.float32, (N,), "bootstrap")
-    te = c.tensor(terminated, torch.uint8, (N, T), "terminated", required=False)
-    tr = c.tensor(truncated, torch.uint8, (N, T), "truncated", required=False)
-    tv = c.tensor(trunc_value, torch.float32, (N, T), "trunc_value", required=tr is not None)
-    out = c.output(returns, torch.float32, (N, T), "returns")
-    st = lib().rlscan_td_lambda(c.ptr(r), c.ptr(v), c.ptr(b), c.ptr(te), c.ptr(tr), c.ptr(tv), c.ptr(out),
+    te = c.tensor(terminated, torch.uint8, S, "terminated", required=False)
+    tr = c.tensor(truncated, torch.uint8, S, "truncated", required=False)
+    tv = c.tensor(trunc_value, torch.float32, S, "trunc_value", required=tr is not None)
+    out = c.output(returns, torch.float32, S, "returns")
+    st = getattr(lib(), name)(c.ptr(r), c.ptr(v), c.ptr(b), c.ptr(te), c.ptr(tr), c.ptr(tv), c.ptr(out),
                                 N, T, float(gamma), float(lam), c.stream(stream))
     return c.finish(st, (out,))[0]
 
 
 def rlscan_discounted_return(rewards, bootstrap=None, terminated=None, truncated=None,
-                             trunc_value=None, *, gamma=0.99, returns=None, stream=None):
+                             trunc_value=None, *, gamma=0.99, returns=None, stream=None, _tm=False):
     """Discounted returns (bootstrap optional).  Returns the [N, T] returns."""
-    N, T = _nt(rewards, "rlscan_discounted_return")
-    c = _Call("rlscan_discounted_return", rewards)
-    r = c.tensor(rewards, torch.float32, (N, T), "rewards")
+    name = "rlscan_discounted_return_tm" if _tm else "rlscan_discounted_return"
+    N, T = _nt(rewards, name, _tm)
+    S = (T, N) if _tm else (N, T)
+    c = _Call(name, rewards)
+    r = c.tensor(rewards, torch.float32, S, "rewards")
     b = c.tensor(bootstrap, torch.float32, (N,), "bootstrap", required=False)
-    te = c.tensor(terminated, torch.uint8, (N, T), "terminated", required=False)
-    tr = c.tensor(truncated, torch.uint8, (N, T), "truncated", required=False)
-    tv = c.tensor(trunc_value, torch.float32, (N, T), "trunc_value", required=tr is not None)
-    out = c.output(returns, torch.float32, (N, T), "returns")
-    st = lib().rlscan_discounted_return(c.ptr(r), c.ptr(b), c.ptr(te), c.ptr(tr), c.ptr(tv), c.ptr(out),
+    te = c.tensor(terminated, torch.uint8, S, "terminated", required=False)
+    tr = c.tensor(truncated, torch.uint8, S, "truncated", required=False)
+    tv = c.tensor(trunc_value, torch.float32, S, "trunc_value", required=tr is not None)
+    out = c.output(returns, torch.float32, S, "returns")
+    st = getattr(lib(), name)(c.ptr(r), c.ptr(b), c.ptr(te), c.ptr(tr), c.ptr(tv), c.ptr(out),
                                         N, T, float(gamma), c.stream(stream))
     return c.finish(st, (out,))[0]
 
 
 def rlscan_elig_trace(inputs, init_trace=None, terminated=None, truncated=None, *, gamma=0.99,
-                      lam=0.95, traces=None, stream=None):
+                      lam=0.95, traces=None, stream=None, _tm=False):
     """Accumulating eligibility traces (forward in time).  Returns the [N, T] traces."""
-    N, T = _nt(inputs, "rlscan_elig_trace")
-    c = _Call("rlscan_elig_trace", inputs)
-    g = c.tensor(inputs, torch.float32, (N, T), "inputs")
+    name = "rlscan_elig_trace_tm" if _tm else "rlscan_elig_trace"
+    N, T = _nt(inputs, name, _tm)
+    S = (T, N) if _tm else (N, T)
+    c = _Call(name, inputs)
+    g = c.tensor(inputs, torch.float32, S, "inputs")
     e0 = c.tensor(init_trace, torch.float32, (N,), "init_trace", required=False)
-    te = c.tensor(terminated, torch.uint8, (N, T), "terminated", required=False)
-    tr = c.tensor(truncated, torch.uint8, (N, T), "truncated", required=False)
-    out = c.output(traces, torch.float32, (N, T), "traces")
-    st = lib().rlscan_elig_trace(c.ptr(g), c.ptr(e0), c.ptr(te), c.ptr(tr), c.ptr(out), N, T,
+    te = c.tensor(terminated, torch.uint8, S, "terminated", required=False)
+    tr = c.tensor(truncated, torch.uint8, S, "truncated", required=False)
+    out = c.output(traces, torch.float32, S, "traces")
+    st = getattr(lib(), name)(c.ptr(g), c.ptr(e0), c.ptr(te), c.ptr(tr), c.ptr(out), N, T,
                                  float(gamma), float(lam), c.stream(stream))
     return c.finish(st, (out,))[0]
 
 
-def rlscan_episodic_prefix_sum(x, terminated=None, truncated=None, *, out=None, stream=None):
+def rlscan_episodic_prefix_sum(x, terminated=None, truncated=None, *, out=None, stream=None, _tm=False):
     """Episodic inclusive prefix sums of int32 values.  Returns the [N, T] int32 sums."""
-    N, T = _nt(x, "rlscan_episodic_prefix_sum")
-    c = _Call("rlscan_episodic_prefix_sum", x)
-    xx = c.tensor(x, torch.int32, (N, T), "x")
-    te = c.tensor(terminated, torch.uint8, (N, T), "terminated", required=False)
-    tr = c.tensor(truncated, torch.uint8, (N, T), "truncated", required=False)
-    o = c.output(out, torch.int32, (N, T), "out")
-    st = lib().rlscan_episodic_prefix_sum(c.ptr(xx), c.ptr(te), c.ptr(tr), c.ptr(o), N, T,
+    name = "rlscan_episodic_prefix_sum_tm" if _tm else "rlscan_episodic_prefix_sum"
+    N, T = _nt(x, name, _tm)
+    S = (T, N) if _tm else (N, T)
+    c = _Call(name, x)
+    xx = c.tensor(x, torch.int32, S, "x")
+    te = c.tensor(terminated, torch.uint8, S, "terminated", required=False)
+    tr = c.tensor(truncated, torch.uint8, S, "truncated", required=False)
+    o = c.output(out, torch.int32, S, "out")
+    st = getattr(lib(), name)(c.ptr(xx), c.ptr(te), c.ptr(tr), c.ptr(o), N, T,
                                           c.stream(stream))
     return c.finish(st, (o,))[0]
 
 
-def rlscan_affine_scan(a, b, reset=None, init=None, *, reverse=False, x=None, stream=None):
+def rlscan_affine_scan(a, b, reset=None, init=None, *, reverse=False, x=None, stream=None, _tm=False):
     """Generic affine scan x_t = b_t + a_t x_prev along T (backward when
     `reverse`), x_prev = init[n] at the row's first step, x_t = b_t where
     reset.  Returns the [N, T] float32 x."""
-    N, T = _nt(a, "rlscan_affine_scan")
-    c = _Call("rlscan_affine_scan", a)
-    aa = c.tensor(a, torch.float32, (N, T), "a")
-    bb = c.tensor(b, torch.float32, (N, T), "b")
-    rs = c.tensor(reset, torch.uint8, (N, T), "reset", required=False)
+    name = "rlscan_affine_scan_tm" if _tm else "rlscan_affine_scan"
+    N, T = _nt(a, name, _tm)
+    S = (T, N) if _tm else (N, T)
+    c = _Call(name, a)
+    aa = c.tensor(a, torch.float32, S, "a")
+    bb = c.tensor(b, torch.float32, S, "b")
+    rs = c.tensor(reset, torch.uint8, S, "reset", required=False)
     x0 = c.tensor(init, torch.float32, (N,), "init", required=False)
-    out = c.output(x, torch.float32, (N, T), "x")
-    st = lib().rlscan_affine_scan(c.ptr(aa), c.ptr(bb), c.ptr(rs), c.ptr(x0), c.ptr(out), N, T,
+    out = c.output(x, torch.float32, S, "x")
+    st = getattr(lib(), name)(c.ptr(aa), c.ptr(bb), c.ptr(rs), c.ptr(x0), c.ptr(out), N, T,
                                   1 if reverse else 0, c.stream(stream))
     return c.finish(st, (out,))[0]
 
@@ -364,6 +389,46 @@ def rlscan_affine_scan_grad(a, x, dy, reset=None, init=None, *, reverse=False, n
 # status, options, plans
 # ---------------------------------------------------------------------------
 
+# ---------------------------------------------------------------------------
+# time-major [T, N] variants: same arguments and results, every per-step
+# tensor [T, N] (per-environment tensors stay [N])
+# ---------------------------------------------------------------------------
+
+def rlscan_gae_tm(*args, **kw):
+    """rlscan_gae on time-major [T, N] tensors.  Returns (advantages, returns or None)."""
+    return rlscan_gae(*args, _tm=True, **kw)
+
+
+def rlscan_vtrace_tm(*args, **kw):
+    """rlscan_vtrace on time-major [T, N] tensors.  Returns (vs, pg or None)."""
+    return rlscan_vtrace(*args, _tm=True, **kw)
+
+
+def rlscan_td_lambda_tm(*args, **kw):
+    """rlscan_td_lambda on time-major [T, N] tensors."""
+    return rlscan_td_lambda(*args, _tm=True, **kw)
+
+
+def rlscan_discounted_return_tm(*args, **kw):
+    """rlscan_discounted_return on time-major [T, N] tensors."""
+    return rlscan_discounted_return(*args, _tm=True, **kw)
+
+
+def rlscan_elig_trace_tm(*args, **kw):
+    """rlscan_elig_trace on time-major [T, N] tensors."""
+    return rlscan_elig_trace(*args, _tm=True, **kw)
+
+
+def rlscan_episodic_prefix_sum_tm(*args, **kw):
+    """rlscan_episodic_prefix_sum on time-major [T, N] tensors."""
+    return rlscan_episodic_prefix_sum(*args, _tm=True, **kw)
+
+
+def rlscan_affine_scan_tm(*args, **kw):
+    """rlscan_affine_scan on time-major [T, N] tensors."""
+    return rlscan_affine_scan(*args, _tm=True, **kw)
+
+
 def rlscan_sync_status(stream=None, raise_on_error=False):
     """Synchronize the stream and return (and clear) the device-side status code."""
     s = torch.cuda.current_stream() if stream is None else stream
@@ -398,6 +463,14 @@ def rlscan_query_plan(estimator: str, N: int, T: int, A: int = 1) -> dict:
     st = lib().rlscan_query_plan(ESTIMATOR_IDS[estimator], int(N), int(T), int(A), ctypes.byref(info))
     if st != 0:
         raise RlscanError("rlscan_query_plan", st)
+    return {f: getattr(info, f) for f, _ in PlanInfo._fields_}
+
+
+def rlscan_query_plan_tm(estimator: str, N: int, T: int) -> dict:
+    info = PlanInfo()
+    st = lib().rlscan_query_plan_tm(ESTIMATOR_IDS[estimator], int(N), int(T), ctypes.byref(info))
+    if st != 0:
+        raise RlscanError("rlscan_query_plan_tm", st)
     return {f: getattr(info, f) for f, _ in PlanInfo._fields_}
 
 

@@ -21,6 +21,7 @@
 #include "retrace.cuh"
 #include "scan_core.cuh"
 #include "scan_kernel.cuh"
+#include "tm_kernel.cuh"
 
 using namespace rlscan;
 
@@ -457,6 +458,74 @@ T *adv(T *p, int64_t elems) {
   return p ? p + elems : nullptr;
 }
 
+// ---------------------------------------------------------------------------
+// time-major [T, N] plans (tm_kernel.cuh)
+// ---------------------------------------------------------------------------
+constexpr int64_t kMaxTmEnvs = int64_t(1) << 26;  // keeps K N inside 32-bit offsets
+
+// Every time-major kernel scans 8 steps per thread (16 kept too many
+// registers live across the look-back).
+using TmGaeOp = GaeOpT<8>;
+using TmVtraceOp = VtraceOpT<8>;
+using TmTdLambdaOp = TdLambdaOpT<8>;
+using TmDiscountedOp = DiscountedOpT<8>;
+using TmEligOp = EligOpT<8>;
+using TmPrefixSumOp = PrefixSumOpT<8>;
+template <bool BWD>
+using TmAffineOp = AffineOp<BWD, float, 8>;
+constexpr int kTmTile = 8;
+
+struct TmPlan {
+  uint32_t wt_log2 = 0, nct = 0, nbc = 0, nchunks = 0, dpitch = 0;
+  size_t ws_bytes = 0;
+};
+
+// Time slices per block: the fewest (a power of two, at most 8) whose K-step
+// tiles cover T, so short windows put more environments in a block.  With
+// forced look-back, the most slices whose span stays below T (when T > K).
+bool make_tm_plan(int K, int64_t N, int64_t T, TmPlan &pl) {
+  if (N > kMaxTmEnvs || T > kMaxRowSteps) return false;
+  uint32_t wl = 0;
+  if (g_force_lookback.load() != 0) {
+    while (wl < 3 && (int64_t(K) << (wl + 1)) < T) ++wl;
+  } else {
+    while (wl < 3 && (int64_t(K) << wl) < T) ++wl;
+  }
+  const int64_t span = int64_t(K) << wl, cols = int64_t(256) >> wl;
+  const int64_t nct = (T + span - 1) / span, nbc = (N + cols - 1) / cols;
+  if (nct * nbc >= (int64_t(1) << 31)) return false;
+  pl.wt_log2 = wl;
+  pl.nct = uint32_t(nct);
+  pl.nbc = uint32_t(nbc);
+  pl.nchunks = uint32_t(nct * nbc);
+  pl.dpitch = uint32_t(nbc * cols);
+  pl.ws_bytes = sizeof(LookbackHeader) + (nct > 1 ? size_t(nct) * size_t(pl.dpitch) * sizeof(LookbackDesc) : 0);
+  return true;
+}
+
+// One launch over the whole [T, N] problem: a block per chunk.
+template <class Op>
+rlscan_status run_tm(const TmPlan &pl, int64_t N, int64_t T, const typename Op::Args &a, rlscan_stream_t stream) {
+  void *ws = nullptr;
+  rlscan_status st = get_workspace(stream, pl.ws_bytes, &ws);
+  if (st != RLSCAN_OK) return st;
+  TmGeom g{};
+  g.N = uint32_t(N);
+  g.T = uint32_t(T);
+  g.wt_log2 = pl.wt_log2;
+  g.nct = pl.nct;
+  g.nbc = pl.nbc;
+  g.nchunks = pl.nchunks;
+  g.dpitch = pl.dpitch;
+  g.lb.hdr = static_cast<LookbackHeader *>(ws);
+  g.lb.desc = reinterpret_cast<LookbackDesc *>(static_cast<LookbackHeader *>(ws) + 1);
+  g.lb.timeout_ns = uint64_t(std::max<int64_t>(1000, g_timeout_ns.load()));
+  g.lb.starve = g_starve.load() != 0 ? 1u : 0u;
+  cudaError_t e = launch(tm_scan_kernel<Op>, pl.nchunks, kTmBlock, 0, stream, a, g);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e == cudaSuccess ? RLSCAN_OK : RLSCAN_ERR_LAUNCH;
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -807,6 +876,187 @@ rlscan_status rlscan_affine_scan_grad(const float *a, const float *x, const floa
         vec);
   };
   return reverse ? go(AffineGradOp<true>{}) : go(AffineGradOp<false>{});
+}
+
+// ---------------------------------------------------------------------------
+// time-major entry points: every per-step array is [T, N] (element (t, n) at
+// t * N + n); per-environment arrays stay [N].  Same checks and results as
+// the row-major calls.
+// ---------------------------------------------------------------------------
+rlscan_status rlscan_gae_tm(const float *rewards, const float *values, const float *bootstrap,
+                            const uint8_t *terminated, const uint8_t *truncated, const float *trunc_value,
+                            float *advantages, float *returns, int64_t N, int64_t T, float gamma, float lambda,
+                            rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  TmPlan pl;
+  if (!make_tm_plan(kTmTile, N, T, pl)) return RLSCAN_ERR_INVALID_ARG;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(rewards), c.need(values), c.need(bootstrap), c.need(advantages);
+  if (truncated) c.need(trunc_value);
+  c.finite(gamma), c.finite(lambda);
+  c.input(rewards, nt * 4, 4), c.input(values, nt * 4, 4), c.input(bootstrap, size_t(N) * 4, 4);
+  c.input(terminated, nt, 1), c.input(truncated, nt, 1);
+  if (truncated) c.input(trunc_value, nt * 4, 4);
+  c.output(advantages, nt * 4, 4), c.output(returns, nt * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  const TmGaeOp::Args a{rewards, values, bootstrap, truncated ? trunc_value : nullptr, terminated, truncated,
+                      advantages, returns, gamma, gamma * lambda};
+  return run_tm<TmGaeOp>(pl, N, T, a, stream);
+}
+
+rlscan_status rlscan_vtrace_tm(const float *log_rhos, const float *rewards, const float *values,
+                               const float *bootstrap, const uint8_t *terminated, const uint8_t *truncated,
+                               const float *trunc_value, float *vs, float *pg_advantages, int64_t N, int64_t T,
+                               float gamma, float lambda, float rho_bar, float c_bar, rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  TmPlan pl;
+  if (!make_tm_plan(kTmTile, N, T, pl)) return RLSCAN_ERR_INVALID_ARG;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(log_rhos), c.need(rewards), c.need(values), c.need(bootstrap), c.need(vs);
+  if (truncated) c.need(trunc_value);
+  c.finite(gamma), c.finite(lambda), c.positive(rho_bar), c.positive(c_bar);
+  c.input(log_rhos, nt * 4, 4), c.input(rewards, nt * 4, 4), c.input(values, nt * 4, 4);
+  c.input(bootstrap, size_t(N) * 4, 4), c.input(terminated, nt, 1), c.input(truncated, nt, 1);
+  if (truncated) c.input(trunc_value, nt * 4, 4);
+  c.output(vs, nt * 4, 4), c.output(pg_advantages, nt * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  const TmVtraceOp::Args a{log_rhos, rewards, values, bootstrap, truncated ? trunc_value : nullptr, terminated,
+                         truncated, vs, pg_advantages, gamma, lambda, rho_bar, c_bar};
+  return run_tm<TmVtraceOp>(pl, N, T, a, stream);
+}
+
+rlscan_status rlscan_td_lambda_tm(const float *rewards, const float *values, const float *bootstrap,
+                                  const uint8_t *terminated, const uint8_t *truncated, const float *trunc_value,
+                                  float *returns, int64_t N, int64_t T, float gamma, float lambda,
+                                  rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  TmPlan pl;
+  if (!make_tm_plan(kTmTile, N, T, pl)) return RLSCAN_ERR_INVALID_ARG;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(rewards), c.need(values), c.need(bootstrap), c.need(returns);
+  if (truncated) c.need(trunc_value);
+  c.finite(gamma), c.finite(lambda);
+  c.input(rewards, nt * 4, 4), c.input(values, nt * 4, 4), c.input(bootstrap, size_t(N) * 4, 4);
+  c.input(terminated, nt, 1), c.input(truncated, nt, 1);
+  if (truncated) c.input(trunc_value, nt * 4, 4);
+  c.output(returns, nt * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  const TmTdLambdaOp::Args a{rewards,  values,  bootstrap, truncated ? trunc_value : nullptr,
+                           terminated, truncated, returns, gamma, gamma * lambda, gamma * (1.0f - lambda)};
+  return run_tm<TmTdLambdaOp>(pl, N, T, a, stream);
+}
+
+rlscan_status rlscan_discounted_return_tm(const float *rewards, const float *bootstrap, const uint8_t *terminated,
+                                          const uint8_t *truncated, const float *trunc_value, float *returns,
+                                          int64_t N, int64_t T, float gamma, rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  TmPlan pl;
+  if (!make_tm_plan(kTmTile, N, T, pl)) return RLSCAN_ERR_INVALID_ARG;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(rewards), c.need(returns);
+  if (truncated) c.need(trunc_value);
+  c.finite(gamma);
+  c.input(rewards, nt * 4, 4), c.input(bootstrap, size_t(N) * 4, 4);
+  c.input(terminated, nt, 1), c.input(truncated, nt, 1);
+  if (truncated) c.input(trunc_value, nt * 4, 4);
+  c.output(returns, nt * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  const TmDiscountedOp::Args a{rewards, bootstrap, truncated ? trunc_value : nullptr, terminated, truncated, returns,
+                             gamma};
+  return run_tm<TmDiscountedOp>(pl, N, T, a, stream);
+}
+
+rlscan_status rlscan_elig_trace_tm(const float *inputs, const float *init_trace, const uint8_t *terminated,
+                                   const uint8_t *truncated, float *traces, int64_t N, int64_t T, float gamma,
+                                   float lambda, rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  TmPlan pl;
+  if (!make_tm_plan(kTmTile, N, T, pl)) return RLSCAN_ERR_INVALID_ARG;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(inputs), c.need(traces);
+  c.finite(gamma), c.finite(lambda);
+  c.input(inputs, nt * 4, 4), c.input(init_trace, size_t(N) * 4, 4);
+  c.input(terminated, nt, 1), c.input(truncated, nt, 1);
+  c.output(traces, nt * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  const TmEligOp::Args a{inputs, init_trace, terminated, truncated, traces, gamma * lambda};
+  return run_tm<TmEligOp>(pl, N, T, a, stream);
+}
+
+rlscan_status rlscan_episodic_prefix_sum_tm(const int32_t *x, const uint8_t *terminated, const uint8_t *truncated,
+                                            int32_t *out, int64_t N, int64_t T, rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  TmPlan pl;
+  if (!make_tm_plan(kTmTile, N, T, pl)) return RLSCAN_ERR_INVALID_ARG;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(x), c.need(out);
+  c.input(x, nt * 4, 4), c.input(terminated, nt, 1), c.input(truncated, nt, 1);
+  c.output(out, nt * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  const TmPrefixSumOp::Args a{x, terminated, truncated, out};
+  return run_tm<TmPrefixSumOp>(pl, N, T, a, stream);
+}
+
+rlscan_status rlscan_affine_scan_tm(const float *a, const float *b, const uint8_t *reset, const float *init,
+                                    float *x, int64_t N, int64_t T, int32_t reverse, rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1) || (reverse != 0 && reverse != 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  TmPlan pl;
+  if (!make_tm_plan(kTmTile, N, T, pl)) return RLSCAN_ERR_INVALID_ARG;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(a), c.need(b), c.need(x);
+  c.input(a, nt * 4, 4), c.input(b, nt * 4, 4), c.input(reset, nt, 1), c.input(init, size_t(N) * 4, 4);
+  c.output(x, nt * 4, 4);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  if (reverse) return run_tm<TmAffineOp<true>>(pl, N, T, TmAffineOp<true>::Args{a, b, init, reset, nullptr, x}, stream);
+  return run_tm<TmAffineOp<false>>(pl, N, T, TmAffineOp<false>::Args{a, b, init, reset, nullptr, x}, stream);
+}
+
+rlscan_status rlscan_query_plan_tm(rlscan_estimator est, int64_t N, int64_t T, rlscan_plan_info *info) {
+  if (!info || !dims_ok(N, T, 1)) return RLSCAN_ERR_INVALID_ARG;
+  switch (est) {
+    case RLSCAN_EST_GAE: case RLSCAN_EST_VTRACE: case RLSCAN_EST_TD_LAMBDA: case RLSCAN_EST_DISCOUNTED_RETURN:
+    case RLSCAN_EST_ELIG_TRACE: case RLSCAN_EST_EPISODIC_PREFIX_SUM: case RLSCAN_EST_AFFINE_SCAN: break;
+    default: return RLSCAN_ERR_INVALID_ARG;
+  }
+  std::memset(info, 0, sizeof(*info));
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  TmPlan pl;
+  if (!make_tm_plan(kTmTile, N, T, pl)) return RLSCAN_ERR_INVALID_ARG;
+  info->block_threads = kTmBlock;
+  info->chunk_steps = int32_t((int64_t(kTmTile) << pl.wt_log2) * (int64_t(256) >> pl.wt_log2));
+  info->lookback = pl.nct > 1 ? 1 : 0;
+  info->launches = 1;
+  info->chunks = pl.nchunks;
+  info->workspace_bytes = int64_t(pl.ws_bytes);
+  return RLSCAN_OK;
 }
 
 rlscan_status rlscan_sync_status(rlscan_stream_t stream) {

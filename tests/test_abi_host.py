@@ -206,3 +206,47 @@ def test_affine_scan_bf16_argument_checks(L):
     assert L.rlscan_affine_scan_bf16(a, b, None, None, P(BASE + 0x20001), 4, 8, 0, None) == INVALID  # odd address
     assert L.rlscan_affine_scan_bf16(a, b, None, None, b, 4, 8, 0, None) == OVERLAP
     assert slr.rlscan_query_plan("affine_scan_bf16", 4096, 2048)["lookback"] == 0
+
+
+def test_time_major_argument_checks(L):
+    r, v, b, o = P(BASE), P(BASE + 0x10000), P(BASE + 0x20000), P(BASE + 0x30000)
+    te = P(BASE + 0x40000)
+    assert L.rlscan_gae_tm(None, None, None, None, None, None, None, None, 0, 5, 0.99, 0.95, None) == OK
+    assert L.rlscan_gae_tm(r, v, b, te, None, None, o, None, -1, 5, 0.99, 0.95, None) == INVALID
+    assert L.rlscan_gae_tm(r, None, b, te, None, None, o, None, 4, 5, 0.99, 0.95, None) == INVALID
+    assert L.rlscan_gae_tm(r, v, b, te, te, None, o, None, 4, 5, 0.99, 0.95, None) == INVALID  # trunc_value
+    assert L.rlscan_gae_tm(r, v, b, te, None, None, r, None, 4, 5, 0.99, 0.95, None) == OVERLAP
+    assert L.rlscan_gae_tm(r, v, b, te, None, None, P(BASE + 0x30002), None, 4, 5, 0.99, 0.95,
+                           None) == INVALID  # misaligned
+    assert L.rlscan_gae_tm(r, v, b, te, None, None, o, None, (1 << 26) + 1, 2, 0.99, 0.95,
+                           None) == INVALID  # more environments than the layout takes
+    assert L.rlscan_vtrace_tm(r, v, b, o, te, None, None, P(BASE + 0x50000), None, 4, 5, 0.99, 1.0, 0.0, 1.0,
+                              None) == INVALID  # rho_bar
+    assert L.rlscan_td_lambda_tm(r, v, b, te, None, None, o, 4, 5, float("nan"), 0.95, None) == INVALID
+    assert L.rlscan_discounted_return_tm(None, None, te, None, None, o, 4, 5, 0.99, None) == INVALID
+    assert L.rlscan_elig_trace_tm(r, None, te, None, r, 4, 5, 0.99, 0.95, None) == OVERLAP
+    assert L.rlscan_episodic_prefix_sum_tm(r, te, None, None, 4, 5, None) == INVALID
+    assert L.rlscan_affine_scan_tm(r, v, None, None, o, 4, 8, 2, None) == INVALID  # direction
+
+
+def test_query_plan_time_major(L):
+    # T <= 64: one chunk per column block of 256 / slices environments
+    for T, cols in [(1, 256), (8, 256), (9, 128), (16, 128), (17, 64), (32, 64), (33, 32), (64, 32)]:
+        p = slr.rlscan_query_plan_tm("gae", 1000, T)
+        assert p["lookback"] == 0 and p["block_threads"] == 256 and p["launches"] == 1
+        assert p["chunks"] == -(-1000 // cols), (T, p)
+    # longer windows chain 64-step chunks of 32 environments
+    p = slr.rlscan_query_plan_tm("vtrace", 4096, 2048)
+    assert p["lookback"] == 1 and p["chunk_steps"] == 64 * 32 and p["chunks"] == 32 * 128
+    assert p["workspace_bytes"] == 16 + 16 * 32 * 4096
+    assert slr.rlscan_query_plan_tm("elig_trace", 33, 65)["chunks"] == 2 * 2
+    # forced look-back halves the chunk while it stays below T
+    slr.rlscan_set_option("force_lookback", 1)
+    try:
+        p = slr.rlscan_query_plan_tm("gae", 100, 32)
+        assert p["lookback"] == 1 and p["chunks"] == 2  # 16-step chunks of 128 environments
+    finally:
+        slr.rlscan_set_option("force_lookback", 0)
+    with pytest.raises(slr.RlscanError):
+        slr.rlscan_query_plan_tm("retrace", 8, 8)
+    assert slr.rlscan_query_plan_tm("affine_scan", 0, 5)["chunks"] == 0

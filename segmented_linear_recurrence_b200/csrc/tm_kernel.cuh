@@ -16,11 +16,12 @@
 // 8 / WT column groups (WT = 1, 2, 4 or 8, the smallest that covers T, at
 // most 8), so a block's chunk is WT K steps of 256 / WT environments.  Inside
 // the chunk the slices' aggregates combine through shared memory; along T,
-// chunks hand carries on with a decoupled look-back per environment: one lane
-// per environment publishes its chunk's aggregate and walks its own
-// predecessors.  Chunks take tickets in dependency order, the column blocks
-// of one time chunk after another, so a block only ever waits on blocks that
-// drew earlier tickets.
+// chunks hand carries on with a decoupled look-back per environment: the
+// chunk's composite is published per environment, and all warps of the block
+// fetch the descriptors of the chunks before it at once, a window of several
+// chunks per memory round trip.  Chunks take tickets in dependency order, the
+// column blocks of one time chunk after another, so a block only ever waits
+// on blocks that drew earlier tickets.
 //
 // Each estimator's coefficients are exactly the row-major kernel's
 // (estimators.cuh, Op::coef); only its loads and stores are restated here
@@ -79,41 +80,71 @@ __device__ __forceinline__ uint32_t ld_na(const uint8_t *p) {
   return v;
 }
 
+// Full tiles (every step valid, the common case) take the unpredicated path.
+template <int K>
+__device__ __forceinline__ bool col_full(const ColTile &c) {
+  return c.valid == (K == 32 ? 0xffffffffu : (1u << K) - 1u);
+}
 template <int K>
 __device__ __forceinline__ void ld_col(const float *p, const ColTile &c, float (&v)[K]) {
   const float *q = p + c.off;
+  if (col_full<K>(c)) {
 #pragma unroll
-  for (int k = 0; k < K; ++k) v[k] = ((c.valid >> k) & 1u) ? ld_na(q + uint32_t(k) * c.N) : 0.0f;
+    for (int k = 0; k < K; ++k) v[k] = ld_na(q + uint32_t(k) * c.N);
+  } else {
+#pragma unroll
+    for (int k = 0; k < K; ++k) v[k] = ((c.valid >> k) & 1u) ? ld_na(q + uint32_t(k) * c.N) : 0.0f;
+  }
 }
 template <int K>
 __device__ __forceinline__ void ld_col(const int32_t *p, const ColTile &c, uint32_t (&v)[K]) {
   const int32_t *q = p + c.off;
+  if (col_full<K>(c)) {
 #pragma unroll
-  for (int k = 0; k < K; ++k) v[k] = ((c.valid >> k) & 1u) ? ld_na(q + uint32_t(k) * c.N) : 0u;
+    for (int k = 0; k < K; ++k) v[k] = ld_na(q + uint32_t(k) * c.N);
+  } else {
+#pragma unroll
+    for (int k = 0; k < K; ++k) v[k] = ((c.valid >> k) & 1u) ? ld_na(q + uint32_t(k) * c.N) : 0u;
+  }
 }
 template <int K>
 __device__ __forceinline__ uint32_t ld_col_flags(const uint8_t *p, const ColTile &c) {
   if (p == nullptr) return 0u;
   const uint8_t *q = p + c.off;
   uint32_t m = 0;
+  if (col_full<K>(c)) {
 #pragma unroll
-  for (int k = 0; k < K; ++k)
-    if (((c.valid >> k) & 1u) && ld_na(q + uint32_t(k) * c.N) != 0u) m |= 1u << k;
+    for (int k = 0; k < K; ++k) m |= (ld_na(q + uint32_t(k) * c.N) != 0u ? 1u : 0u) << k;
+  } else {
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+      if (((c.valid >> k) & 1u) && ld_na(q + uint32_t(k) * c.N) != 0u) m |= 1u << k;
+  }
   return m;
 }
 template <int K>
 __device__ __forceinline__ void st_col(float *p, const ColTile &c, const float (&v)[K]) {
   float *q = p + c.off;
+  if (col_full<K>(c)) {
 #pragma unroll
-  for (int k = 0; k < K; ++k)
-    if ((c.valid >> k) & 1u) __stcs(q + uint32_t(k) * c.N, v[k]);
+    for (int k = 0; k < K; ++k) __stcs(q + uint32_t(k) * c.N, v[k]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+      if ((c.valid >> k) & 1u) __stcs(q + uint32_t(k) * c.N, v[k]);
+  }
 }
 template <int K>
 __device__ __forceinline__ void st_col(int32_t *p, const ColTile &c, const uint32_t (&v)[K]) {
   int32_t *q = p + c.off;
+  if (col_full<K>(c)) {
 #pragma unroll
-  for (int k = 0; k < K; ++k)
-    if ((c.valid >> k) & 1u) __stcs(q + uint32_t(k) * c.N, int(v[k]));
+    for (int k = 0; k < K; ++k) __stcs(q + uint32_t(k) * c.N, int(v[k]));
+  } else {
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+      if ((c.valid >> k) & 1u) __stcs(q + uint32_t(k) * c.N, int(v[k]));
+  }
 }
 
 // Done flag (terminated or truncated) of the step before the tile.
@@ -320,90 +351,72 @@ struct TmIO<AffineOp<BWD, float, K>> {
 };
 
 // ---------------------------------------------------------------------------
-// Look-back along T for one environment per lane.  Descriptor (chunk j,
-// environment n) sits at j * dpitch + n, so a warp's 32 descriptors of one
-// chunk are contiguous.  The lane publishes its chunk's aggregate (its final
-// value at once if the aggregate cuts), then walks the chunks its carry
-// depends on (j + 1, j + 2, ... backward; j - 1, j - 2, ... forward), loading
-// D descriptors per round trip and composing aggregates in dependency order
-// until it meets a final one: an inclusive value, or an aggregate that cuts
-// (a = 0, which the window-edge chunk always is).  Waits are bounded by
-// `timeout_ns` of global time and an iteration cap; on expiry the lane
-// records the timeout status, takes the partial carry and still publishes.
-// The protocol is scan_core.cuh's: self-validating 64-bit words tagged with
-// the launch's epoch, no fences.
+// Look-back along T, one environment per lane, the whole block fetching.
+// Descriptor (chunk j, environment n) sits at j * dpitch + n, so a warp's 32
+// descriptors of one chunk are contiguous; the protocol is scan_core.cuh's
+// (self-validating 64-bit words tagged with the launch's epoch, no fences).
+// In each round every warp of a column group fetches kTmWin descriptors per
+// lane, so the group's WT warps see WT kTmWin chunks in one memory round
+// trip; each thread polls its own until ready (bounded by timeout_ns of
+// global time and an iteration cap), combines them in dependency order up to
+// the first final one (an inclusive value, an aggregate that cuts, or the
+// array end) and posts that one entry to shared memory.  After a barrier the
+// group's publishing warp walks the WT entries in dependency order; columns
+// still open fetch the next window.
 // ---------------------------------------------------------------------------
-template <bool BACKWARD, typename V, int D = 2>
-__device__ V column_lookback(const LookbackCtl &ctl, uint32_t j, uint32_t nct, uint32_t dpitch, uint32_t n,
-                             bool active, uint32_t epoch, uint32_t ticket, Aff<V> agg, bool edge_closed) {
-  const uint32_t tag = epoch << 2;
-  const bool silent = ctl.starve && ticket == 0;
-  LookbackDesc *mine = ctl.desc + size_t(j) * dpitch + n;
-  const bool self_cut = cuts(agg);
-  if (active && !silent) {
-    if (self_cut) {
-      st_relaxed_u64(&mine->w[0], desc_word(tag | kDescInclusive, to_bits(agg.b)));
-    } else {
-      st_relaxed_u64(&mine->w[1], desc_word(tag | kDescAggregate, to_bits(agg.b)));
-      st_relaxed_u64(&mine->w[0], desc_word(tag | kDescAggregate, to_bits(agg.a)));
+constexpr int kTmWin = 2;  // descriptors per thread per round
+enum : uint32_t { kWinAggregate = 0, kWinFinal = 1 };
+
+template <typename V>
+struct TmWindow {
+  uint32_t state[kTmBlock / 32][32];  // per fetching thread: its kTmWin descriptors combined
+  V a[kTmBlock / 32][32], b[kTmBlock / 32][32];
+  V cin[kTmBlock / 32][32];           // [column group][lane]: carry entering the chunk
+  uint32_t open[kTmBlock / 32][32];   // [column group][lane]: walk not finished
+};
+
+// Decodes a descriptor's two words: false if not ready yet, else the entry
+// (state, a, b): an aggregate, or a final value in b.
+template <typename V>
+__device__ __forceinline__ bool decode_desc(unsigned long long w0, unsigned long long w1, uint32_t tag,
+                                            uint32_t &st, V &a, V &b) {
+  const uint32_t f0 = uint32_t(w0 >> 32);
+  if (f0 == (tag | kDescInclusive)) {
+    st = kWinFinal;
+    b = from_bits<V>(uint32_t(w0));
+    return true;
+  }
+  if (f0 == (tag | kDescAggregate) && uint32_t(w1 >> 32) == (tag | kDescAggregate)) {
+    a = from_bits<V>(uint32_t(w0));
+    b = from_bits<V>(uint32_t(w1));
+    st = cuts(Aff<V>{a, b}) ? kWinFinal : kWinAggregate;  // an aggregate that cuts carries its own value
+    return true;
+  }
+  return false;
+}
+
+// Polls a descriptor whose first read was not ready until it is, bounded by
+// limit_ns of global time from t0 and an iteration cap; on expiry it records
+// the timeout status and returns a final 0, so the walk ends with the partial
+// carry.
+template <typename V>
+__device__ __forceinline__ void wait_desc(const LookbackDesc *d, uint32_t tag, uint32_t t0, uint32_t limit_ns,
+                                       uint32_t &st, V &a, V &b) {
+  const uint32_t max_polls = 64u + limit_ns / 32u;
+  uint32_t sleep_ns = 16u;
+  for (uint32_t polls = 0;; ++polls) {
+    __nanosleep(sleep_ns);
+    sleep_ns = min(sleep_ns * 2u, 256u);
+    unsigned long long w0, w1;
+    ld_relaxed_desc(d, w0, w1);
+    if (decode_desc<V>(w0, w1, tag, st, a, b)) return;
+    if (polls > max_polls || uint32_t(global_timer_ns()) - t0 > limit_ns) {
+      record_status(kDevStatusTimeout);
+      st = kWinFinal;
+      b = V(0);
+      return;
     }
   }
-  V carry = V(0);
-  if (active && !edge_closed) {
-    Aff<V> acc = aff_identity<V>();
-    int32_t q = BACKWARD ? int32_t(j) + 1 : int32_t(j) - 1;  // nearest chunk not yet composed
-    const uint32_t t0 = uint32_t(global_timer_ns());
-    const uint32_t limit_ns = uint32_t(min(ctl.timeout_ns, uint64_t(1) << 31));
-    const uint32_t max_polls = 64u + limit_ns / 32u;
-    uint32_t polls = 0, sleep_ns = 0;
-    for (;;) {
-      unsigned long long w0[D], w1[D];
-#pragma unroll
-      for (int d = 0; d < D; ++d) {
-        const int32_t qd = BACKWARD ? q + d : q - d;
-        w0[d] = w1[d] = 0ull;
-        if (qd >= 0 && uint32_t(qd) < nct) ld_relaxed_desc(ctl.desc + size_t(qd) * dpitch + n, w0[d], w1[d]);
-      }
-      int used = 0;
-      bool done = false;
-#pragma unroll
-      for (int d = 0; d < D; ++d) {
-        if (!done && used == d) {
-          const int32_t qd = BACKWARD ? q + d : q - d;
-          const uint32_t f0 = uint32_t(w0[d] >> 32);
-          if (qd < 0 || uint32_t(qd) >= nct) {  // past the array end: nothing enters
-            carry = acc.b;
-            done = true;
-          } else if (f0 == (tag | kDescInclusive)) {
-            carry = apply(acc, from_bits<V>(uint32_t(w0[d])));
-            done = true;
-          } else if (f0 == (tag | kDescAggregate) && uint32_t(w1[d] >> 32) == (tag | kDescAggregate)) {
-            const Aff<V> e{from_bits<V>(uint32_t(w0[d])), from_bits<V>(uint32_t(w1[d]))};
-            acc = compose(acc, e);
-            used = d + 1;
-            if (cuts(e)) {  // an aggregate that cuts carries its own value
-              carry = acc.b;
-              done = true;
-            }
-          }
-        }
-      }
-      if (done) break;
-      q = BACKWARD ? q + used : q - used;
-      if (used == 0) {
-        if (++polls > max_polls || uint32_t(global_timer_ns()) - t0 > limit_ns) {
-          record_status(kDevStatusTimeout);
-          carry = acc.b;
-          break;
-        }
-        if (sleep_ns) __nanosleep(sleep_ns);
-        sleep_ns = sleep_ns ? min(sleep_ns * 2u, 256u) : 16u;
-      }
-    }
-  }
-  if (active && !silent && !self_cut)
-    st_relaxed_u64(&mine->w[0], desc_word(tag | kDescInclusive, to_bits(apply(agg, carry))));
-  return carry;
 }
 
 // Registers per thread of the time-major kernels, and the blocks per SM that
@@ -428,7 +441,6 @@ __global__ void __launch_bounds__(kTmBlock, tm_min_blocks())
   constexpr uint32_t kFull = K == 32 ? 0xffffffffu : (1u << K) - 1u;
 
   __shared__ Aff<V> s_agg[kTmBlock / 32][32];    // [warp][lane]: each thread's K-step composite
-  __shared__ V s_carry[kTmBlock / 32][32];       // [column group][lane]: carry entering the chunk
   __shared__ uint32_t s_ticket, s_epoch;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -521,14 +533,85 @@ __global__ void __launch_bounds__(kTmBlock, tm_min_blocks())
   V cin = V(0);
   if (lb) {
     // a7: the slice farthest from the chunk's dependency edge holds the
-    // chunk's composite once its own is added; its warp runs the look-back.
-    if (slice == (BWD ? 0u : wt - 1u)) {
-      const bool closed = BWD ? (j == g.nct - 1u) : (j == 0u);
-      s_carry[group][lane] = column_lookback<BWD, V>(g.lb, j, g.nct, g.dpitch, c.n, col_ok, epoch, ticket,
-                                                     compose(agg, pre), closed);
+    // chunk's composite once its own is added, and publishes it.
+    __shared__ TmWindow<V> s_win;
+    const uint32_t tag = epoch << 2;
+    const bool silent = g.lb.starve && ticket == 0;
+    const bool owner = slice == (BWD ? 0u : wt - 1u);
+    const Aff<V> tot = compose(agg, pre);
+    LookbackDesc *mine = g.lb.desc + size_t(j) * g.dpitch + c.n;
+    if (owner && col_ok && !silent) {
+      if (cuts(tot)) {
+        st_relaxed_u64(&mine->w[0], desc_word(tag | kDescInclusive, to_bits(tot.b)));
+      } else {
+        st_relaxed_u64(&mine->w[1], desc_word(tag | kDescAggregate, to_bits(tot.b)));
+        st_relaxed_u64(&mine->w[0], desc_word(tag | kDescAggregate, to_bits(tot.a)));
+      }
     }
-    __syncthreads();
-    cin = s_carry[group][lane];
+    const uint32_t limit_ns = uint32_t(min(g.lb.timeout_ns, uint64_t(1) << 31));
+    const uint32_t per_round = wt * uint32_t(kTmWin);
+    Aff<V> acc = aff_identity<V>();  // publishing warp: composite walked so far
+    bool open = col_ok && !(BWD ? (j == g.nct - 1u) : (j == 0u));
+    const bool walked = open;  // the column needs a carry (else it enters 0)
+    for (uint32_t base = 1u;; base += per_round) {
+      // Fetch this round's window, chunk distances base + slice kTmWin + d:
+      // every load goes out before any is waited on.
+      if (open) {
+        const uint32_t t0 = uint32_t(global_timer_ns());
+        unsigned long long w0[kTmWin], w1[kTmWin];
+#pragma unroll
+        for (int d = 0; d < kTmWin; ++d) {
+          const uint32_t dist = base + slice * uint32_t(kTmWin) + uint32_t(d);
+          w0[d] = w1[d] = 0ull;
+          if (BWD ? (dist < g.nct - j) : (dist <= j))
+            ld_relaxed_desc(g.lb.desc + size_t(BWD ? j + dist : j - dist) * g.dpitch + c.n, w0[d], w1[d]);
+        }
+        uint32_t est = kWinAggregate;
+        Aff<V> e = aff_identity<V>();
+#pragma unroll
+        for (int d = 0; d < kTmWin; ++d) {
+          if (est == kWinAggregate) {
+            const uint32_t dist = base + slice * uint32_t(kTmWin) + uint32_t(d);
+            uint32_t st = kWinFinal;  // past the array end: nothing enters
+            V ea = V(1), eb = V(0);
+            if (BWD ? (dist < g.nct - j) : (dist <= j)) {
+              if (!decode_desc<V>(w0[d], w1[d], tag, st, ea, eb))
+                wait_desc<V>(g.lb.desc + size_t(BWD ? j + dist : j - dist) * g.dpitch + c.n, tag, t0, limit_ns,
+                             st, ea, eb);
+            }
+            if (st == kWinFinal) {
+              e = Aff<V>{V(0), apply(e, eb)};
+              est = kWinFinal;
+            } else {
+              e = compose(e, Aff<V>{ea, eb});
+            }
+          }
+        }
+        s_win.state[warp][lane] = est;
+        s_win.a[warp][lane] = e.a;
+        s_win.b[warp][lane] = e.b;
+      }
+      __syncthreads();
+      // The publishing warp walks the group's window in dependency order.
+      if (owner && open) {
+        for (uint32_t u = 0; u < wt; ++u) {
+          const Aff<V> e{s_win.a[w0 + u][lane], s_win.b[w0 + u][lane]};
+          if (s_win.state[w0 + u][lane] == kWinFinal) {
+            cin = apply(acc, e.b);
+            open = false;
+            break;
+          }
+          acc = compose(acc, e);
+        }
+        s_win.cin[group][lane] = cin;
+        s_win.open[group][lane] = open ? 1u : 0u;
+      }
+      if (!__syncthreads_or(owner && open)) break;
+      if (!owner && open) open = s_win.open[group][lane] != 0u;
+    }
+    if (!owner && walked) cin = s_win.cin[group][lane];
+    if (owner && col_ok && !silent && !cuts(tot))
+      st_relaxed_u64(&mine->w[0], desc_word(tag | kDescInclusive, to_bits(apply(tot, cin))));
   }
 
   // a8: re-sweep from the carry entering the tile, then the outputs.

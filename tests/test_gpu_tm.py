@@ -140,9 +140,10 @@ def test_time_major_host_tensors():
     assert_parity("gae", tuple(np.ascontiguousarray(g.T) for g in got), ref, what="host tensors")
 
 
-def test_time_major_unaligned_views():
+@pytest.mark.parametrize("N", [37, 64])
+def test_time_major_unaligned_views(N):
     # Views one element into a larger buffer: 4-byte aligned, not 16.
-    N, T = 37, 301
+    T = 301
     d = inputs("td_lambda", N, T, seed=3500)
     s = f32_scalars("td_lambda", synthetic.SCALARS["td_lambda"])
     dt = transpose(d)

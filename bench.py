@@ -215,22 +215,38 @@ def workload_calls(workload: str, rank: int):
     return calls
 
 
+def time_major(workload: str) -> bool:
+    return synthetic.WORKLOADS[workload].get("layout") == "time_major"
+
+
+def call_arrays(est, d, tm):
+    """The call's input arrays in argument order, time-major when `tm`."""
+    dd = synthetic.to_time_major(d) if tm else d
+    return [dd.get(k) for k in ARG_ORDER[est]]
+
+
+def call_plan(slr, est, d, T, tm):
+    A = d["q"].shape[2] if est == "retrace" else 1
+    N = d["q"].shape[0] if est == "retrace" else d[ARG_ORDER[est][0]].shape[0]
+    return slr.rlscan_query_plan_tm(est, N, T) if tm else slr.rlscan_query_plan(est, N, T, A)
+
+
 class DeviceCall:
-    def __init__(self, est, T, d, device):
+    def __init__(self, est, T, d, device, tm=False):
         import torch
-        self.est, self.T = est, T
-        self.inputs = [None if d.get(k) is None else torch.from_numpy(d[k]).to(device)
-                       for k in ARG_ORDER[est]]
+        self.est, self.T, self.tm = est, T, tm
+        self.inputs = [None if a is None else torch.from_numpy(a).to(device) for a in call_arrays(est, d, tm)]
         shape = d["q"].shape[:2] if est == "retrace" else d[ARG_ORDER[est][0]].shape
+        shape = tuple(shape[::-1]) if tm else tuple(shape)
         dt = torch.int32 if est == "episodic_prefix_sum" else torch.float32
-        self.outs = {k: torch.empty(tuple(shape), dtype=dt, device=device) for k in OUT_KW[est]}
+        self.outs = {k: torch.empty(shape, dtype=dt, device=device) for k in OUT_KW[est]}
         self.scal = {} if est == "episodic_prefix_sum" else dict(synthetic.SCALARS[est])
         self.steps = int(np.prod(shape))
         self.bytes = algorithmic_bytes(est, d)
 
     def launch(self):
         import segmented_linear_recurrence_b200 as slr
-        getattr(slr, f"rlscan_{self.est}")(*self.inputs, **self.scal, **self.outs)
+        getattr(slr, f"rlscan_{self.est}{'_tm' if self.tm else ''}")(*self.inputs, **self.scal, **self.outs)
 
 
 def run_gpu(args, rank, world, local_rank):
@@ -246,13 +262,12 @@ def run_gpu(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(device)
 
     host_calls = workload_calls(args.workload, rank)
-    calls = [DeviceCall(est, T, d, device) for est, T, d in host_calls]
+    tm = time_major(args.workload)
+    calls = [DeviceCall(est, T, d, device, tm) for est, T, d in host_calls]
     steps_per_step = sum(c.steps for c in calls)
     launches_per_step = 0
     for est, T, d in host_calls:
-        A = d["q"].shape[2] if est == "retrace" else 1
-        N = d["q"].shape[0] if est == "retrace" else d[ARG_ORDER[est][0]].shape[0]
-        launches_per_step += slr.rlscan_query_plan(est, N, T, A)["launches"]
+        launches_per_step += call_plan(slr, est, d, T, tm)["launches"]
 
     def eager_step():
         for c in calls:
@@ -263,9 +278,7 @@ def run_gpu(args, rank, world, local_rank):
     cap_stream = torch.cuda.Stream(device)
     ws = 0
     for est, T, d in host_calls:
-        A = d["q"].shape[2] if est == "retrace" else 1
-        N = d["q"].shape[0] if est == "retrace" else d[ARG_ORDER[est][0]].shape[0]
-        ws = max(ws, slr.rlscan_query_plan(est, N, T, A)["workspace_bytes"])
+        ws = max(ws, call_plan(slr, est, d, T, tm)["workspace_bytes"])
     slr.rlscan_reserve_workspace(ws, cap_stream)
     warm_done = 0
     with torch.cuda.stream(cap_stream):
@@ -359,18 +372,19 @@ def run_e2e(args, host_calls, device, world):
     import segmented_linear_recurrence_b200 as slr
     pinned = []
     h2d = d2h = 0
+    tm = time_major(args.workload)
     for est, T, d in host_calls:
-        ins = [None if d.get(k) is None else torch.from_numpy(d[k]).pin_memory() for k in ARG_ORDER[est]]
+        ins = [None if a is None else torch.from_numpy(a).pin_memory() for a in call_arrays(est, d, tm)]
         h2d += sum(x.numel() * x.element_size() for x in ins if x is not None)
         shape = d["q"].shape[:2] if est == "retrace" else d[ARG_ORDER[est][0]].shape
         d2h += 4 * int(np.prod(shape)) * len(OUT_KW[est])
         scal = {} if est == "episodic_prefix_sum" else dict(synthetic.SCALARS[est])
-        pinned.append((est, ins, scal))
+        pinned.append((f"rlscan_{est}{'_tm' if tm else ''}", ins, scal))
 
     def step():
         out = None
-        for est, ins, scal in pinned:
-            out = getattr(slr, f"rlscan_{est}")(*ins, **scal)
+        for fn, ins, scal in pinned:
+            out = getattr(slr, fn)(*ins, **scal)
         return out
 
     step()  # warm the caching allocators
@@ -457,21 +471,28 @@ def run_reference(args):
 def run_one(args):
     """`--one EST N T [A]`: `--steps` plain calls of one estimator on seeded
     inputs of the workload recipe (p_term 0.02, p_trunc 0.005 where the
-    estimator takes truncation), for ncu captures of a single kernel."""
+    estimator takes truncation), for ncu captures of a single kernel.  EST
+    with a `_tm` suffix runs the time-major entry point."""
     import torch
     import segmented_linear_recurrence_b200 as slr
     from segmented_linear_recurrence_b200 import build as slr_build
     slr_build.build()
     est, N, T = args.one[0], int(args.one[1]), int(args.one[2])
+    tm = est.endswith("_tm")
+    est = est[:-3] if tm else est
     A = int(args.one[3]) if len(args.one) > 3 else 18
     trunc = 0.0 if est in ("retrace", "elig_trace", "episodic_prefix_sum") else 0.005
-    d = synthetic.make_inputs(est, N, T, seed=5, p_term=0.02, p_trunc=trunc, A=A, with_init=True)
-    call = DeviceCall(est, T, d, torch.device("cuda", 0))
+    if est == "affine_scan":
+        d = synthetic.make_affine_inputs(N, T, seed=5, p_reset=0.02)
+    else:
+        d = synthetic.make_inputs(est, N, T, seed=5, p_term=0.02, p_trunc=trunc, A=A, with_init=True)
+    call = DeviceCall(est, T, d, torch.device("cuda", 0), tm)
     for _ in range(max(args.steps, 1)):
         call.launch()
     torch.cuda.synchronize()
     st = slr.rlscan_sync_status()
-    print(json.dumps({"one": est, "N": N, "T": T, "A": A, "calls": args.steps, "status": st}))
+    print(json.dumps({"one": est + ("_tm" if tm else ""), "N": N, "T": T, "A": A, "calls": args.steps,
+                      "status": st}))
     return 0 if st == 0 else 1
 
 
@@ -529,8 +550,9 @@ def main():
     dom = max(per_est, key=lambda k: per_est[k]["ms"])
     de = per_est[dom]
     achieved = de["bytes"] / (de["ms"] / 1000.0) / 1e9
-    dom_kernel = f"scan_kernel<{dom}>"
-    traffic = load_traffic(dom)
+    tm = time_major(args.workload)
+    dom_kernel = f"tm_scan_kernel<{dom}>" if tm else f"scan_kernel<{dom}>"
+    traffic = None if tm else load_traffic(dom)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "kernel": dom_kernel, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
@@ -551,6 +573,7 @@ def main():
         "config": {"workload": args.workload, "estimators": list(w["estimators"]),
                    "N_envs_per_gpu": w["N"], "T": list(w["Ts"]), "p_term": w["p_term"],
                    "p_trunc": w["p_trunc"], "calls_per_step": len(calls),
+                   "layout": "time-major [T, N]" if tm else "row-major [N, T]",
                    "l2": "inputs > L2: every call reads its own buffers; "
                          f"{sum(sum(x.numel() * x.element_size() for x in c.inputs if x is not None) for c in calls) / 1e9:.2f}"
                          " GB of distinct inputs per step",

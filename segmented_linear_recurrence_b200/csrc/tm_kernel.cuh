@@ -194,6 +194,7 @@ struct TmIO;
 template <int K>
 struct TmIO<GaeOpT<K>> {
   using Op = GaeOpT<K>;
+  static constexpr int kRegs = 64;  // registers per thread, chosen by measurement
   static __device__ __forceinline__ void load(const typename Op::Args &p, const ColTile &c, Flags f,
                                               typename Op::Raw &w) {
     ld_col(p.r, c, w.r);
@@ -222,6 +223,7 @@ struct TmIO<GaeOpT<K>> {
 template <int K>
 struct TmIO<TdLambdaOpT<K>> {
   using Op = TdLambdaOpT<K>;
+  static constexpr int kRegs = 64;  // registers per thread, chosen by measurement
   static __device__ __forceinline__ void load(const typename Op::Args &p, const ColTile &c, Flags f,
                                               typename Op::Raw &w) {
     ld_col(p.r, c, w.r);
@@ -244,6 +246,7 @@ struct TmIO<TdLambdaOpT<K>> {
 template <int K>
 struct TmIO<DiscountedOpT<K>> {
   using Op = DiscountedOpT<K>;
+  static constexpr int kRegs = 48;  // registers per thread, chosen by measurement
   static __device__ __forceinline__ void load(const typename Op::Args &p, const ColTile &c, Flags f,
                                               typename Op::Raw &w) {
     ld_col(p.r, c, w.r);
@@ -264,6 +267,7 @@ struct TmIO<DiscountedOpT<K>> {
 template <int K>
 struct TmIO<VtraceOpT<K>> {
   using Op = VtraceOpT<K>;
+  static constexpr int kRegs = 64;  // registers per thread, chosen by measurement
   static __device__ __forceinline__ void load(const typename Op::Args &p, const ColTile &c, Flags f,
                                               typename Op::Raw &w) {
     ld_col(p.lr, c, w.lr);
@@ -296,6 +300,7 @@ struct TmIO<VtraceOpT<K>> {
 template <int K>
 struct TmIO<EligOpT<K>> {
   using Op = EligOpT<K>;
+  static constexpr int kRegs = 48;  // registers per thread, chosen by measurement
   static __device__ __forceinline__ void load(const typename Op::Args &p, const ColTile &c, Flags f,
                                               typename Op::Raw &w) {
     ld_col(p.g, c, w.g);
@@ -315,6 +320,7 @@ struct TmIO<EligOpT<K>> {
 template <int K>
 struct TmIO<PrefixSumOpT<K>> {
   using Op = PrefixSumOpT<K>;
+  static constexpr int kRegs = 48;  // registers per thread, chosen by measurement
   static __device__ __forceinline__ void load(const typename Op::Args &p, const ColTile &c, Flags f,
                                               typename Op::Raw &w) {
     ld_col(p.x, c, w.x);
@@ -334,6 +340,7 @@ struct TmIO<PrefixSumOpT<K>> {
 template <bool BWD, int K>
 struct TmIO<AffineOp<BWD, float, K>> {
   using Op = AffineOp<BWD, float, K>;
+  static constexpr int kRegs = 48;  // registers per thread, chosen by measurement
   static __device__ __forceinline__ void load(const typename Op::Args &p, const ColTile &c, Flags f,
                                               typename Op::Raw &w) {
     ld_col(p.a, c, w.a);
@@ -419,20 +426,22 @@ __device__ __forceinline__ void wait_desc(const LookbackDesc *d, uint32_t tag, u
   }
 }
 
-// Registers per thread of the time-major kernels, and the blocks per SM that
-// leaves: a thread's K steps stay live (coefficients and the values its
-// outputs need) across the slice combine and the look-back, which spilled at
-// the row-major kernels' tighter budgets.
-constexpr int kTmRegs = 64;
+// Blocks per SM that the estimator's register budget (TmIO<Op>::kRegs)
+// leaves, over the four 16K-register partitions.  A thread's K steps stay
+// live (coefficients and the values its outputs need) across the slice
+// combine and the look-back: 64 registers for the estimators with two or
+// three per-step inputs, 48 (a few spilled bytes, more blocks resident) for
+// the lighter ones, where it measured faster.
+template <class IO>
 constexpr int tm_min_blocks() {
   constexpr int warps = kTmBlock / 32;
   int b = 2048 / kTmBlock;
-  while (b > 1 && ((b * warps + 3) / 4) * 32 * kTmRegs > 16384) --b;
+  while (b > 1 && ((b * warps + 3) / 4) * 32 * IO::kRegs > 16384) --b;
   return b;
 }
 
 template <class Op>
-__global__ void __launch_bounds__(kTmBlock, tm_min_blocks())
+__global__ void __launch_bounds__(kTmBlock, tm_min_blocks<TmIO<Op>>())
     tm_scan_kernel(const typename Op::Args p, const TmGeom g) {
   using V = typename Op::V;
   using IO = TmIO<Op>;

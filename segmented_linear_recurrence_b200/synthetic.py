@@ -53,7 +53,20 @@ WORKLOADS = {
     # the generic affine scan (backward), resets at p_term
     "affine_4096xT": dict(index=5, N=4096, Ts=(512, 2048), estimators=("affine_scan",), p_term=0.01,
                           p_trunc=0.0),
+    # the sweep's estimators and the affine scan on time-major [T, N] buffers
+    "tm_4096xT": dict(index=6, N=4096, Ts=(512, 2048),
+                      estimators=("gae", "vtrace", "td_lambda", "discounted_return", "affine_scan"),
+                      p_term=0.02, p_trunc=0.005, layout="time_major"),
 }
+
+# Per-environment arrays ([N]) keep their shape in the time-major layout.
+PER_ENV_KEYS = ("bootstrap", "init_trace", "init")
+
+
+def to_time_major(d: dict) -> dict:
+    """The same inputs with every [N, T] array stored time-major [T, N]."""
+    return {k: (None if v is None else (v if k in PER_ENV_KEYS else np.ascontiguousarray(v.T)))
+            for k, v in d.items()}
 
 
 def seed_for(workload: str, estimator: str, T: int) -> int:

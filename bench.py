@@ -93,9 +93,10 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def load_traffic(kernel_key: str):
-    """Per-launch DRAM bytes of a kernel from the committed ncu summary, if it
-    was taken on the current kernel sources (else None)."""
+def load_traffic(workload: str, est: str):
+    """Per-launch DRAM bytes of one estimator's kernel in a workload, from the
+    committed ncu summary, if it was taken on the current kernel sources (else
+    None)."""
     from segmented_linear_recurrence_b200 import build as slr_build
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
@@ -105,7 +106,7 @@ def load_traffic(kernel_key: str):
         return None
     if j.get("source_hash") != slr_build.source_hash():
         return None
-    k = j.get("kernels", {}).get(kernel_key)
+    k = j.get("workloads", {}).get(workload, {}).get("kernels", {}).get(est)
     return None if k is None else k.get("dram_bytes_per_launch")
 
 
@@ -552,7 +553,7 @@ def main():
     achieved = de["bytes"] / (de["ms"] / 1000.0) / 1e9
     tm = time_major(args.workload)
     dom_kernel = f"tm_scan_kernel<{dom}>" if tm else f"scan_kernel<{dom}>"
-    traffic = None if tm else load_traffic(dom)
+    traffic = load_traffic(args.workload, dom)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "kernel": dom_kernel, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",

@@ -552,7 +552,7 @@ def main():
     de = per_est[dom]
     achieved = de["bytes"] / (de["ms"] / 1000.0) / 1e9
     tm = time_major(args.workload)
-    dom_kernel = f"tm_scan_kernel<{dom}>" if tm else f"scan_kernel<{dom}>"
+    dom_kernel = f"tm_scan_kernel<{dom}>" if tm else ("retrace_kernel" if dom == "retrace" else f"scan_kernel<{dom}>")
     traffic = load_traffic(args.workload, dom)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,

@@ -105,6 +105,22 @@ rlscan_status rlscan_gae(const float *rewards, const float *values, const float 
                          int64_t T, float gamma, float lambda, rlscan_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * GAE with bfloat16 I/O (reduced-precision storage; the pages hint at format
+ * limits, gist.science technical summary, Resultaten).  Same arguments
+ * and checks as rlscan_gae, but every real array -- rewards, values,
+ * bootstrap, trunc_value, advantages, returns -- holds bfloat16 values
+ * (passed as their uint16_t bit patterns, 2-byte aligned).  The arithmetic is
+ * fp32: inputs widen exactly, the scan runs in fp32, and each output is
+ * rounded to the nearest bfloat16 (ties to even), so it differs from rlscan_gae
+ * on the widened inputs by at most one rounding to 8 significant bits (2^-8
+ * relative) plus the fp32 scan error.  9 bytes per step instead of 17.
+ * ------------------------------------------------------------------------- */
+rlscan_status rlscan_gae_bf16(const uint16_t *rewards, const uint16_t *values, const uint16_t *bootstrap,
+                              const uint8_t *terminated, const uint8_t *truncated, const uint16_t *trunc_value,
+                              uint16_t *advantages, uint16_t *returns, int64_t N, int64_t T, float gamma,
+                              float lambda, rlscan_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * GAE without any device allocation.  The paper has no counterpart: this is a
  * deployment variant of rlscan_gae for callers that must not allocate device
  * memory -- for example code that runs while its stream is being captured
@@ -340,7 +356,8 @@ typedef enum rlscan_estimator {
   RLSCAN_EST_EPISODIC_PREFIX_SUM = 6,
   RLSCAN_EST_AFFINE_SCAN = 7,
   RLSCAN_EST_AFFINE_SCAN_GRAD = 8,
-  RLSCAN_EST_AFFINE_SCAN_BF16 = 9
+  RLSCAN_EST_AFFINE_SCAN_BF16 = 9,
+  RLSCAN_EST_GAE_BF16 = 10
 } rlscan_estimator;
 
 /* How a call of the given shape is executed (no device work, no allocation). */

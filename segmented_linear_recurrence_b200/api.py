@@ -26,7 +26,7 @@ __all__ = [
     "rlscan_abi_version", "rlscan_query_plan", "rlscan_set_option", "rlscan_get_option",
     "rlscan_reserve_workspace", "rlscan_gae_tm", "rlscan_vtrace_tm", "rlscan_td_lambda_tm",
     "rlscan_discounted_return_tm", "rlscan_elig_trace_tm", "rlscan_episodic_prefix_sum_tm",
-    "rlscan_affine_scan_tm", "rlscan_query_plan_tm",
+    "rlscan_affine_scan_tm", "rlscan_query_plan_tm", "rlscan_gae_bf16",
     "STATUS", "OPTIONS", "ESTIMATOR_IDS", "LIB_PATH",
 ]
 
@@ -39,7 +39,7 @@ OPTIONS = {"lookback_timeout_ns": 1, "force_lookback": 2, "force_block": 3, "for
            "check_pointers": 5, "test_starve_lookback": 6, "pdl": 7}
 ESTIMATOR_IDS = {"gae": 0, "vtrace": 1, "retrace": 2, "td_lambda": 3, "discounted_return": 4,
                  "elig_trace": 5, "episodic_prefix_sum": 6, "affine_scan": 7, "affine_scan_grad": 8,
-                 "affine_scan_bf16": 9}
+                 "affine_scan_bf16": 9, "gae_bf16": 10}
 
 
 class RlscanError(RuntimeError):
@@ -67,6 +67,7 @@ _SIGNATURES = {
     "rlscan_affine_scan": [_VP] * 5 + [_I64, _I64, ctypes.c_int32, _VP],
     "rlscan_affine_scan_grad": [_VP] * 8 + [_I64, _I64, ctypes.c_int32, _VP],
     "rlscan_affine_scan_bf16": [_VP] * 5 + [_I64, _I64, ctypes.c_int32, _VP],
+    "rlscan_gae_bf16": [_VP] * 8 + [_I64, _I64, _F, _F, _VP],
     "rlscan_gae_tm": [_VP] * 8 + [_I64, _I64, _F, _F, _VP],
     "rlscan_vtrace_tm": [_VP] * 9 + [_I64, _I64, _F, _F, _F, _F, _VP],
     "rlscan_td_lambda_tm": [_VP] * 7 + [_I64, _I64, _F, _F, _VP],
@@ -348,6 +349,25 @@ def rlscan_affine_scan(a, b, reset=None, init=None, *, reverse=False, x=None, st
     st = getattr(lib(), name)(c.ptr(aa), c.ptr(bb), c.ptr(rs), c.ptr(x0), c.ptr(out), N, T,
                                   1 if reverse else 0, c.stream(stream))
     return c.finish(st, (out,))[0]
+
+
+def rlscan_gae_bf16(rewards, values, bootstrap, terminated=None, truncated=None, trunc_value=None, *,
+                    gamma=0.99, lam=0.95, advantages=None, returns=None, want_returns=True, stream=None):
+    """rlscan_gae on bfloat16 tensors (fp32 arithmetic, bf16 results).
+    Returns (advantages, returns or None)."""
+    N, T = _nt(rewards, "rlscan_gae_bf16")
+    c = _Call("rlscan_gae_bf16", rewards)
+    r = c.tensor(rewards, torch.bfloat16, (N, T), "rewards")
+    v = c.tensor(values, torch.bfloat16, (N, T), "values")
+    b = c.tensor(bootstrap, torch.bfloat16, (N,), "bootstrap")
+    te = c.tensor(terminated, torch.uint8, (N, T), "terminated", required=False)
+    tr = c.tensor(truncated, torch.uint8, (N, T), "truncated", required=False)
+    tv = c.tensor(trunc_value, torch.bfloat16, (N, T), "trunc_value", required=tr is not None)
+    adv = c.output(advantages, torch.bfloat16, (N, T), "advantages")
+    ret = c.output(returns, torch.bfloat16, (N, T), "returns") if (want_returns or returns is not None) else None
+    st = lib().rlscan_gae_bf16(c.ptr(r), c.ptr(v), c.ptr(b), c.ptr(te), c.ptr(tr), c.ptr(tv), c.ptr(adv),
+                               c.ptr(ret), N, T, float(gamma), float(lam), c.stream(stream))
+    return c.finish(st, (adv, ret))
 
 
 def rlscan_affine_scan_bf16(a, b, reset=None, init=None, *, reverse=False, x=None, stream=None):

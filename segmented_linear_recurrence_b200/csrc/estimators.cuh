@@ -219,8 +219,8 @@ struct Flags {
 // row's bootstrap at a row end (`boot` may be NULL: 0); termination wins over
 // truncation, and both over the row end.  trunc_value is the only load whose
 // address depends on loaded data; warps without a truncated step skip it.
-template <int K>
-__device__ __forceinline__ void boundary_successors(const float *tv, const float *boot, float ev, const Tile &tl,
+template <int K, class E = float>
+__device__ __forceinline__ void boundary_successors(const E *tv, const E *boot, float ev, const Tile &tl,
                                                     Flags f, const FastDiv &fd, float (&bv)[K]) {
   const uint32_t tr = f.trunc & ~f.term & tl.valid;
   const uint32_t ed = tl.edge & ~f.term & ~f.trunc;
@@ -229,29 +229,31 @@ __device__ __forceinline__ void boundary_successors(const float *tv, const float
   if (__any_sync(0xffffffffu, tr != 0u)) {
 #pragma unroll
     for (int k = 0; k < K; ++k)
-      if ((tr >> k) & 1u) bv[k] = __ldg(tv + tl.i0 + k);
+      if ((tr >> k) & 1u) bv[k] = ld1(tv + tl.i0 + k);
   }
   if (ed != 0u) {  // at most one row end per tile when T >= 8
 #pragma unroll
     for (int k = 0; k < K; ++k)
-      if ((ed >> k) & 1u) bv[k] = tl.few_rows ? ev : (boot ? __ldg(boot + tl.n0 + fd.div(tl.t0 + k)) : 0.0f);
+      if ((ed >> k) & 1u) bv[k] = tl.few_rows ? ev : (boot ? ld1(boot + tl.n0 + fd.div(tl.t0 + k)) : 0.0f);
   }
 }
 
 // ---------------------------------------------------------------------------
 // GAE (Schulman et al. 2016): x = advantage, a = gamma lambda cont,
-// b = r + gamma nv - v.  Outputs advantages = x, returns = x + v.
+// b = r + gamma nv - v.  Outputs advantages = x, returns = x + v.  E is the
+// storage type of every real array: float, or __nv_bfloat16 (bf16 I/O, fp32
+// arithmetic, outputs rounded to nearest even).
 // ---------------------------------------------------------------------------
-template <int K_ = kTile>
+template <int K_ = kTile, class E = float>
 struct GaeOpT {
   static constexpr int K = K_;  // steps per thread
   static constexpr int kRegs = 48, kRegsLookback = 48;  // registers per thread, chosen by measurement
   using V = float;
   static constexpr bool kBackward = true;
   struct Args {
-    const float *r, *v, *boot, *tv;
+    const E *r, *v, *boot, *tv;
     const uint8_t *term, *trunc;
-    float *adv, *ret;
+    E *adv, *ret;
     float gamma, gl;
   };
   struct Raw {
@@ -265,11 +267,11 @@ struct GaeOpT {
     ld_tile(p.r, tl, w.r);
     ld_tile(p.v, tl, w.v);
     w.f = f;
-    w.halo = (lane == 31 && tl.nvalid == K && tl.i0 + uint32_t(K) < total) ? __ldg(p.v + tl.i0 + uint32_t(K)) : 0.0f;
+    w.halo = (lane == 31 && tl.nvalid == K && tl.i0 + uint32_t(K) < total) ? ld1(p.v + tl.i0 + uint32_t(K)) : 0.0f;
     w.ev = edge_value(p.boot, tl, fd);
   }
   static __device__ __forceinline__ void fetch_boundary(const Args &p, const Tile &tl, const FastDiv &fd, Raw &w) {
-    boundary_successors(p.tv, p.boot, w.ev, tl, w.f, fd, w.bv);
+    boundary_successors<K, E>(p.tv, p.boot, w.ev, tl, w.f, fd, w.bv);
   }
   static __device__ __forceinline__ float nbr_of(const Raw &w) { return w.v[0]; }
   static __device__ __forceinline__ float halo_of(const Raw &w) { return w.halo; }

@@ -240,6 +240,8 @@ int64_t rows_per_block(int64_t T, int block, int64_t tile) {
   return k;
 }
 
+using GaeBf16Op = GaeOpT<kTile, __nv_bfloat16>;  // GAE with bf16 I/O
+
 // Steps per thread of each estimator's kernel (Op::K).
 int tile_steps(rlscan_estimator est) {
   switch (est) {
@@ -252,6 +254,7 @@ int tile_steps(rlscan_estimator est) {
     case RLSCAN_EST_AFFINE_SCAN: return AffineOp<false>::K;
     case RLSCAN_EST_AFFINE_SCAN_GRAD: return AffineGradOp<false>::K;
     case RLSCAN_EST_AFFINE_SCAN_BF16: return AffineOp<false, __nv_bfloat16>::K;
+    case RLSCAN_EST_GAE_BF16: return GaeBf16Op::K;
     default: return 4;  // Retrace: its own 4-step tiles
   }
 }
@@ -566,6 +569,45 @@ rlscan_status rlscan_gae(const float *rewards, const float *values, const float 
         return aligned(adv(rewards, o), 32) && aligned(adv(values, o), 32) &&
                aligned(adv(advantages, o), 32) && aligned(adv(returns, o), 32) &&
                aligned(adv(terminated, o), 8) && aligned(adv(truncated, o), 8);
+      });
+}
+
+rlscan_status rlscan_gae_bf16(const uint16_t *rewards, const uint16_t *values, const uint16_t *bootstrap,
+                              const uint8_t *terminated, const uint8_t *truncated, const uint16_t *trunc_value,
+                              uint16_t *advantages, uint16_t *returns, int64_t N, int64_t T, float gamma,
+                              float lambda, rlscan_stream_t stream) {
+  if (!dims_ok(N, T, 1)) return RLSCAN_ERR_INVALID_ARG;
+  if (N == 0 || T == 0) return RLSCAN_OK;
+  const size_t nt = size_t(N) * size_t(T);
+  Checker c;
+  c.need(rewards), c.need(values), c.need(bootstrap), c.need(advantages);
+  if (truncated) c.need(trunc_value);
+  c.finite(gamma), c.finite(lambda);
+  c.input(rewards, nt * 2, 2), c.input(values, nt * 2, 2), c.input(bootstrap, size_t(N) * 2, 2);
+  c.input(terminated, nt, 1), c.input(truncated, nt, 1);
+  if (truncated) c.input(trunc_value, nt * 2, 2);
+  c.output(advantages, nt * 2, 2), c.output(returns, nt * 2, 2);
+  c.check_overlaps();
+  c.check_device_access(stream);
+  if (c.st != RLSCAN_OK) return c.st;
+  using B16 = __nv_bfloat16;
+  using Op = GaeBf16Op;
+  const Plan pl = make_plan(RLSCAN_EST_GAE_BF16, N, T, 1);
+  auto b16 = [](const uint16_t *p) { return reinterpret_cast<const B16 *>(p); };
+  B16 *advb = reinterpret_cast<B16 *>(advantages), *retb = reinterpret_cast<B16 *>(returns);
+  const B16 *tv = truncated ? b16(trunc_value) : nullptr;
+  return run<Op>(
+      pl, N, T, stream,
+      [&](int64_t r0) {
+        const int64_t o = r0 * T;
+        return Op::Args{adv(b16(rewards), o), adv(b16(values), o), adv(b16(bootstrap), r0), adv(tv, o),
+                        adv(terminated, o),   adv(truncated, o),   adv(advb, o),             adv(retb, o),
+                        gamma,                gamma * lambda};
+      },
+      [&](int64_t r0) {
+        const int64_t o = r0 * T;
+        return aligned(adv(rewards, o), 16) && aligned(adv(values, o), 16) && aligned(adv(advantages, o), 16) &&
+               aligned(adv(returns, o), 16) && aligned(adv(terminated, o), 8) && aligned(adv(truncated, o), 8);
       });
 }
 
@@ -1124,7 +1166,7 @@ int rlscan_abi_version(void) { return RLSCAN_ABI_VERSION; }
 
 rlscan_status rlscan_query_plan(rlscan_estimator est, int64_t N, int64_t T, int64_t A,
                                 rlscan_plan_info *info) {
-  if (!info || int(est) < 0 || int(est) > int(RLSCAN_EST_AFFINE_SCAN_BF16)) return RLSCAN_ERR_INVALID_ARG;
+  if (!info || int(est) < 0 || int(est) > int(RLSCAN_EST_GAE_BF16)) return RLSCAN_ERR_INVALID_ARG;
   if (est != RLSCAN_EST_RETRACE) A = 1;
   if (A < 1 || A > kMaxActions || !dims_ok(N, T, A)) return RLSCAN_ERR_INVALID_ARG;
   std::memset(info, 0, sizeof(*info));

@@ -250,3 +250,13 @@ def test_query_plan_time_major(L):
     with pytest.raises(slr.RlscanError):
         slr.rlscan_query_plan_tm("retrace", 8, 8)
     assert slr.rlscan_query_plan_tm("affine_scan", 0, 5)["chunks"] == 0
+
+
+def test_gae_bf16_argument_checks(L):
+    r, v, b, o = P(BASE), P(BASE + 0x10000), P(BASE + 0x20000), P(BASE + 0x30000)
+    assert L.rlscan_gae_bf16(None, None, None, None, None, None, None, None, 0, 5, 0.99, 0.95, None) == OK
+    assert L.rlscan_gae_bf16(r, v, None, None, None, None, o, None, 4, 8, 0.99, 0.95, None) == INVALID  # bootstrap
+    assert L.rlscan_gae_bf16(r, v, b, None, None, None, P(BASE + 0x30001), None, 4, 8, 0.99, 0.95,
+                             None) == INVALID  # odd address
+    assert L.rlscan_gae_bf16(r, v, b, None, None, None, v, None, 4, 8, 0.99, 0.95, None) == OVERLAP
+    assert L.rlscan_gae_bf16(r, v, b, None, None, None, o, None, 4, 8, float("inf"), 0.95, None) == INVALID

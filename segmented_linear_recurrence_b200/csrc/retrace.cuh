@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(BLOCK) retrace_kernel(const RetraceOp::Args p,
     ticket = s_ticket;
     epoch = s_epoch;
     if (ticket >= g.nchunks) return;  // counter left inconsistent by an aborted launch
-    chunk = g.nchunks - 1u - ticket;
+    chunk = chunk_of_ticket(g, ticket, true);
   }
   uint32_t lo, hi, base;
   if constexpr (LB) {

@@ -438,6 +438,7 @@ rlscan_status run(const Plan &pl, int64_t N, int64_t T, rlscan_stream_t stream, 
     g.nchunks = blocks_in_launch(pl, rows, T);
     g.span = pl.L;
     g.rows_per_chunk = uint32_t(pl.rows_per_block);
+    g.cpr = (pl.lookback && T % int64_t(pl.L) == 0) ? uint32_t(T / int64_t(pl.L)) : 0u;
     const bool vec = g_force_scalar.load() == 0 && slice_vec(r0);
     g.vec = vec ? 1u : 0u;
     fast_div_params(uint32_t(T), g.div_m, g.div_l);
@@ -1287,6 +1288,7 @@ extern "C" rlscan_status rlscan_gae_noalloc(const float *rewards, const float *v
   g.nchunks = blocks_in_launch(pl, N, T);
   g.span = pl.L;
   g.rows_per_chunk = uint32_t(pl.rows_per_block);
+  g.cpr = (pl.lookback && T % int64_t(pl.L) == 0) ? uint32_t(T / int64_t(pl.L)) : 0u;
   g.vec = (g_force_scalar.load() == 0 && aligned(rewards, 32) && aligned(values, 32) && aligned(advantages, 32) &&
            aligned(returns, 32) && aligned(terminated, 8) && aligned(truncated, 8))
               ? 1u

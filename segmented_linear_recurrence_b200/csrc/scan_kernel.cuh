@@ -49,8 +49,24 @@ struct ScanGeom {
   uint32_t rows_per_chunk;  // rows plan: k
   uint32_t vec;           // 1: arrays aligned for 256-bit (flags: 64-bit) accesses
   uint32_t div_m, div_l;  // FastDiv by T
+  uint32_t cpr;           // look-back plan: chunks per row when rows are whole chunks, else 0
   LookbackCtl lb;         // ticket / done / epoch counters and descriptors (look-back only)
 };
+
+// Look-back plan: the chunk a ticket stands for.  Tickets go out in
+// dependency order, so a block only waits on chunks whose tickets were drawn
+// earlier.  When rows are whole chunks (cpr > 0) the tickets interleave the
+// rows -- the first chunk in dependency order of every row, then the second
+// of every row, ... -- so a chunk's predecessor drew its ticket a whole
+// launch's rows earlier and has normally published by the time it is needed;
+// a row's first chunk needs no carry.  Otherwise the flat order: chunks
+// straddle rows and the predecessor is the previous ticket.
+__device__ __forceinline__ uint32_t chunk_of_ticket(const ScanGeom &g, uint32_t ticket, bool backward) {
+  if (g.cpr == 0u) return backward ? g.nchunks - 1u - ticket : ticket;
+  const uint32_t rows = g.nchunks / g.cpr;
+  const uint32_t s = ticket / rows, r = ticket - s * rows;
+  return r * g.cpr + (backward ? g.cpr - 1u - s : s);
+}
 
 // Steps, row position and row edges of the K-step tile at step i0 (a multiple of K)
 // of a block that owns the steps [lo, hi), i0 + 8 > lo.
@@ -320,14 +336,14 @@ __global__ void __launch_bounds__(BLOCK, (min_blocks_per_sm<Op, BLOCK, LB>()))
   grid_dependency_wait();
 
   if constexpr (LB) {
-    // Chunk selection: tickets go out in dependency order (backward: the
-    // highest chunk first), so whatever a block waits for is owned by a
-    // block that has already started.
+    // Chunk selection: tickets go out in dependency order (chunk_of_ticket),
+    // so whatever a block waits for is owned by a block that has already
+    // started.
     if (tid == 0 && !draw_ticket(g.lb.hdr, g.nchunks, sm.ticket, sm.epoch)) record_status(kDevStatusTimeout);
     __syncthreads();
     const uint32_t ticket = sm.ticket;
     if (ticket >= g.nchunks) return;  // counter left inconsistent by an aborted launch
-    const uint32_t chunk = BWD ? g.nchunks - 1u - ticket : ticket;
+    const uint32_t chunk = chunk_of_ticket(g, ticket, BWD);
     const uint32_t lo = chunk * L, hi = min(lo + L, g.total);
     const Tile tl = make_tile<BWD, K>(g, fd, lo + uint32_t(K) * uint32_t(tid), lo, hi);
     const Flags f{ld_flags<K>(p.term, tl), ld_flags<K>(p.trunc, tl)};

@@ -157,3 +157,19 @@ def test_graph_capture_and_replay(est, N, T):
         torch.cuda.synchronize()
         assert_parity(est, tuple(outs[k].cpu().numpy() for k in OUTPUT_NAMES[est]), ref, what="replay")
     assert slr.rlscan_sync_status() == 0
+
+
+# Look-back with rows of whole chunks (T a multiple of the chunk): tickets
+# interleave the rows (every row's first chunk in dependency order, then every
+# row's second, ...).  Mixed with a T whose chunks straddle rows (flat order)
+# for the 16-step estimators.
+@pytest.mark.parametrize("est", synthetic.ESTIMATORS)
+def test_row_interleaved_tickets_match_oracle(est):
+    cases = {"retrace": [(37, 4096), (9, 8192)], "elig_trace": [(37, 16384), (130, 12288), (3, 10000)],
+             "episodic_prefix_sum": [(37, 16384), (130, 12288), (3, 10000)]}.get(
+                 est, [(37, 16384), (130, 8192), (3, 6144)])
+    for N, T in cases:
+        d = synthetic.make_inputs(est, N, T, seed=990 + N + T, p_term=0.002, p_trunc=0.002, A=6,
+                                  with_init=True)
+        assert slr.rlscan_query_plan(est, N, T, 6)["lookback"] == 1
+        check(est, d, synthetic.SCALARS[est], what=f"interleaved N={N} T={T}")

@@ -408,7 +408,7 @@ __device__ __forceinline__ bool decode_desc(unsigned long long w0, unsigned long
 // carry.
 template <typename V>
 __device__ __forceinline__ void wait_desc(const LookbackDesc *d, uint32_t tag, uint32_t t0, uint32_t limit_ns,
-                                       uint32_t &st, V &a, V &b) {
+                                          uint32_t &st, V &a, V &b) {
   const uint32_t max_polls = 64u + limit_ns / 32u;
   uint32_t sleep_ns = 16u;
   for (uint32_t polls = 0;; ++polls) {
@@ -430,8 +430,9 @@ __device__ __forceinline__ void wait_desc(const LookbackDesc *d, uint32_t tag, u
 // leaves, over the four 16K-register partitions.  A thread's K steps stay
 // live (coefficients and the values its outputs need) across the slice
 // combine and the look-back: 64 registers for the estimators with two or
-// three per-step inputs, 48 (a few spilled bytes, more blocks resident) for
-// the lighter ones, where it measured faster.
+// three per-step inputs, 48 (more blocks resident; a few spilled bytes for
+// the eligibility trace and the prefix sum) for the lighter ones, where it
+// measured faster.
 template <class IO>
 constexpr int tm_min_blocks() {
   constexpr int warps = kTmBlock / 32;

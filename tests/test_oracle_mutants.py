@@ -49,6 +49,9 @@ MUTANTS = {
                                   "if (have_next) g += a_next * g_next;"),
     "affine_grad_wrong_neighbour": ("xp = (double)x[n * T + (reverse ? t + 1 : t - 1)];",
                                     "xp = (double)x[n * T + (reverse ? t - 1 : t + 1)];"),
+    "affine_tm_row_major_index": ("const int64_t i = t * N + n;", "const int64_t i = n * T + t;"),
+    "affine_tm_ignores_direction": ("const int64_t t = reverse ? T - 1 - k : k;\n      const int64_t i = t * N + n;",
+                                    "const int64_t t = k;\n      const int64_t i = t * N + n;"),
 }
 
 PIN_TESTS = [
@@ -64,6 +67,8 @@ PIN_TESTS = [
     lambda: pins.test_affine_every_reset_pattern(False),
     lambda: pins.test_affine_grad_matches_finite_differences(False, 0.3),
     lambda: pins.test_affine_grad_matches_finite_differences(True, 0.3),
+    lambda: pins.test_affine_tm_matches_bruteforce_on_transpose(True),
+    lambda: pins.test_affine_tm_is_row_major_on_transposed_arrays(),
 ]
 
 

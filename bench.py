@@ -305,6 +305,32 @@ def run_gpu(args, rank, world, local_rank):
             evs[-1].record(cur)
         return g, evs
 
+    # Concurrent step graph: the workload's calls are independent, so each
+    # estimator's calls run on a stream of their own (fork from and join back
+    # to the capture stream); every stream has its own look-back workspace.
+    ests = list(dict.fromkeys(c.est for c in calls))
+    nstreams = max(1, min(args.streams, len(ests)))
+    side = [torch.cuda.Stream(device) for _ in range(nstreams)] if nstreams > 1 else []
+    for s_ in side:
+        slr.rlscan_reserve_workspace(ws, s_)
+
+    def launch_concurrent(root):
+        for s_ in side:
+            s_.wait_stream(root)
+        for j, c in enumerate(calls):
+            with torch.cuda.stream(side[ests.index(c.est) % nstreams]):
+                c.launch()
+        for s_ in side:
+            root.wait_stream(s_)
+
+    g_conc = None
+    if side:
+        launch_concurrent(cap_stream)  # eager once: each stream's workspace in use before capture
+        torch.cuda.synchronize()
+        g_conc = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_conc, stream=cap_stream):
+            launch_concurrent(torch.cuda.current_stream())
+
     # plain step graph (timed: value), per-estimator-group events (timed:
     # roofline), per-launch events (diagnostic per-T table)
     g_plain, _ = capture([])
@@ -315,8 +341,10 @@ def run_gpu(args, rank, world, local_rank):
     g_group, ev_group = capture(groups)
     g_each, ev_each = capture(list(range(len(calls))))
     while warm_done < max(args.warmup, 1):
-        g_plain.replay()
+        (g_conc or g_plain).replay()
         warm_done += 1
+    if g_conc is not None:
+        g_plain.replay()
     g_group.replay()
     g_each.replay()
     torch.cuda.synchronize()
@@ -344,7 +372,8 @@ def run_gpu(args, rank, world, local_rank):
                             for i in range(len(per_step_events) - 1)])
         return t0.elapsed_time(t1), acc
 
-    elapsed_ms, _ = timed(g_plain)
+    serial_ms, _ = timed(g_plain)
+    elapsed_ms = timed(g_conc)[0] if g_conc is not None else serial_ms
     group_ms_total, group_last = timed(g_group, ev_group)
     clocks = sampler.stop()
     _, each_last = timed(g_each, ev_each)
@@ -354,14 +383,16 @@ def run_gpu(args, rank, world, local_rank):
     group_ms = group_last * (group_ms_total / args.steps) / max(group_last.sum(), 1e-9)
     per_group = {calls[j].est: float(group_ms[i]) for i, j in enumerate(groups)}
     per_call_ms = each_last
-    del g_plain, g_group, g_each
+    del g_plain, g_group, g_each, g_conc
     max_ms = max_over_ranks(elapsed_ms, device)
+    max_serial_ms = max_over_ranks(serial_ms, device)
 
     # e2e: the same step through the public API from pinned host buffers
     e2e = run_e2e(args, host_calls, device, world)
 
     return dict(calls=calls, steps_per_step=steps_per_step, launches_per_step=launches_per_step,
-                elapsed_ms=max_ms, per_call_ms=per_call_ms, per_group=per_group,
+                elapsed_ms=max_ms, serial_ms=max_serial_ms, streams=nstreams, per_call_ms=per_call_ms,
+                per_group=per_group,
                 group_ms_per_step=group_ms_total / args.steps, clocks=clocks, e2e=e2e,
                 warmup=warm_done, status=status)
 
@@ -505,6 +536,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", choices=tuple(synthetic.WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--streams", type=int, default=4,
+                    help="streams the step's independent estimators run on (1: one stream, in order)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU work for the oracle baseline (0 disables it)")
     ap.add_argument("--one", nargs="+", metavar="EST N T [A]",
@@ -579,6 +612,7 @@ def main():
                          f"{sum(sum(x.numel() * x.element_size() for x in c.inputs if x is not None) for c in calls) / 1e9:.2f}"
                          " GB of distinct inputs per step",
                    "timing": "K replays of a CUDA graph holding one step's launches, CUDA events around the K",
+                   "streams": res["streams"],
                    "parallelism": f"dp{world} (independent env shards, no collective)"},
         "roofline": roofline,
         "gpu_launches": int(res["launches_per_step"] * args.steps),
@@ -592,6 +626,8 @@ def main():
                               "ms_per_step": round(v["ms"], 4),
                               "by_T_event_per_launch": v["by_T"]} for k, v in per_est.items()},
         "ms_per_step_with_group_events": res["group_ms_per_step"],
+        "ms_per_step_one_stream": res["serial_ms"] / args.steps,
+        "value_one_stream": aggregate_rate(world, res["steps_per_step"], res["serial_ms"] / args.steps),
         "device_status": res["status"],
     }
     if rank == 0 and world == 1 and args.cpu_seconds > 0:

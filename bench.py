@@ -461,9 +461,48 @@ def cpu_baseline(host_calls, seconds: float):
         if time.perf_counter() - t0 >= seconds:
             break
     dt = time.perf_counter() - t0
-    return {"value": done_steps / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+    line = {"value": done_steps / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{passes} full pass(es) over the workload ({done_steps} env-steps, "
                       f"{dt:.1f} s, one thread, fp64)"}
+    line.update(cpu_baseline_all_cores(host_calls, seconds / 2))
+    return line
+
+
+def cpu_baseline_all_cores(host_calls, seconds: float):
+    """The same oracle on every host core: each call's rows split into one
+    slice per thread (the C loops release the interpreter lock), whole passes
+    until at least `seconds` have run.  Reported beside the one-thread value."""
+    from concurrent.futures import ThreadPoolExecutor
+    import oracle
+    workers = max(1, os.cpu_count() or 1)
+
+    def sliced(d, lo, hi):
+        return {k: (None if v is None else v[lo:hi]) for k, v in d.items()}
+
+    def one_pass(pool):
+        futs, steps = [], 0
+        for est, T, d in host_calls:
+            N = d["q"].shape[0] if est == "retrace" else d[ARG_ORDER[est][0]].shape[0]
+            steps += N * T
+            per = -(-N // workers)
+            for lo in range(0, N, per):
+                futs.append(pool.submit(oracle.run, est, sliced(d, lo, min(N, lo + per)), **synthetic.SCALARS[est]))
+        for f in futs:
+            f.result()
+        return steps
+
+    with ThreadPoolExecutor(max_workers=workers) as pool:
+        one_pass(pool)  # warm
+        done, passes = 0, 0
+        t0 = time.perf_counter()
+        while True:
+            done += one_pass(pool)
+            passes += 1
+            if time.perf_counter() - t0 >= seconds:
+                break
+        dt = time.perf_counter() - t0
+    return {"all_cores_value": done / dt, "all_cores": workers,
+            "all_cores_sample": f"{passes} full pass(es), rows split over {workers} threads, {dt:.1f} s"}
 
 
 def run_reference(args):

@@ -26,7 +26,7 @@ __all__ = [
     "rlscan_abi_version", "rlscan_query_plan", "rlscan_set_option", "rlscan_get_option",
     "rlscan_reserve_workspace", "rlscan_gae_tm", "rlscan_vtrace_tm", "rlscan_td_lambda_tm",
     "rlscan_discounted_return_tm", "rlscan_elig_trace_tm", "rlscan_episodic_prefix_sum_tm",
-    "rlscan_affine_scan_tm", "rlscan_query_plan_tm", "rlscan_gae_bf16",
+    "rlscan_affine_scan_tm", "rlscan_query_plan_tm", "rlscan_gae_bf16", "affine_scan",
     "STATUS", "OPTIONS", "ESTIMATOR_IDS", "LIB_PATH",
 ]
 
@@ -403,6 +403,34 @@ def rlscan_affine_scan_grad(a, x, dy, reset=None, init=None, *, reverse=False, n
     st = lib().rlscan_affine_scan_grad(c.ptr(aa), c.ptr(xx), c.ptr(gy), c.ptr(rs), c.ptr(x0), c.ptr(o_da),
                                        c.ptr(o_db), c.ptr(o_di), N, T, 1 if reverse else 0, c.stream(stream))
     return c.finish(st, (o_da, o_db, o_di))
+
+
+class _AffineScanFn(torch.autograd.Function):
+    """Autograd glue: the forward is rlscan_affine_scan, the backward its adjoint
+    kernel rlscan_affine_scan_grad (nothing is computed here)."""
+
+    @staticmethod
+    def forward(ctx, a, b, init, reset, reverse):
+        x = rlscan_affine_scan(a, b, reset, init, reverse=reverse)
+        ctx.save_for_backward(a, x, init)
+        ctx.reset, ctx.reverse = reset, reverse
+        return x
+
+    @staticmethod
+    def backward(ctx, dy):
+        a, x, init = ctx.saved_tensors
+        need_da, need_db, need_di = ctx.needs_input_grad[0], ctx.needs_input_grad[1], ctx.needs_input_grad[2]
+        if not (need_da or need_db or need_di):
+            return None, None, None, None, None
+        da, db, di = rlscan_affine_scan_grad(a, x, dy.contiguous(), ctx.reset, init, reverse=ctx.reverse,
+                                             need_da=need_da, need_dinit=need_di and init is not None)
+        return (da if need_da else None, db if need_db else None, di if need_di else None, None, None)
+
+
+def affine_scan(a, b, reset=None, init=None, *, reverse=False):
+    """Differentiable rlscan_affine_scan for torch autograd: gradients with
+    respect to a, b and init come from the adjoint scan kernel."""
+    return _AffineScanFn.apply(a, b, init, reset, bool(reverse))
 
 
 # ---------------------------------------------------------------------------

@@ -15,6 +15,7 @@ pinned inputs for asynchronous copies.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 
 import torch
@@ -194,10 +195,34 @@ def _nt(x, name, tm=False):
     return (int(x.shape[1]), int(x.shape[0])) if tm else (int(x.shape[0]), int(x.shape[1]))
 
 
+def _layout_dispatch(fn):
+    """Per-step tensors given as [N, T] views of time-major [T, N] storage
+    (every 2-D argument non-contiguous with a contiguous transpose, as
+    `buf.T` gives) run on the time-major kernel without a copy; the outputs
+    come back as [N, T] views of time-major buffers."""
+    def is2d(x):
+        return isinstance(x, torch.Tensor) and x.dim() == 2
+
+    @functools.wraps(fn)
+    def wrapper(*args, **kw):
+        if kw.get("_tm"):
+            return fn(*args, **kw)
+        mats = [x for x in list(args) + list(kw.values()) if is2d(x)]
+        if mats and all(not x.is_contiguous() and x.t().is_contiguous() for x in mats):
+            res = fn(*[x.t() if is2d(x) else x for x in args], _tm=True,
+                     **{k: (v.t() if is2d(v) else v) for k, v in kw.items()})
+            if isinstance(res, tuple):
+                return tuple(None if r is None else r.t() for r in res)
+            return res.t()
+        return fn(*args, **kw)
+    return wrapper
+
+
 # ---------------------------------------------------------------------------
 # estimators
 # ---------------------------------------------------------------------------
 
+@_layout_dispatch
 def rlscan_gae(rewards, values, bootstrap, terminated=None, truncated=None, trunc_value=None, *,
                gamma=0.99, lam=0.95, advantages=None, returns=None, want_returns=True, stream=None, _tm=False):
     """GAE advantages and returns.  Returns (advantages, returns or None)."""
@@ -218,6 +243,7 @@ def rlscan_gae(rewards, values, bootstrap, terminated=None, truncated=None, trun
     return c.finish(st, (adv, ret))
 
 
+@_layout_dispatch
 def rlscan_vtrace(log_rhos, rewards, values, bootstrap, terminated=None, truncated=None,
                   trunc_value=None, *, gamma=0.99, lam=1.0, rho_bar=1.0, c_bar=1.0, vs=None,
                   pg_advantages=None, want_pg=True, stream=None, _tm=False):
@@ -264,6 +290,7 @@ def rlscan_retrace(q, pi, mu_a, actions, rewards, bootstrap, terminated=None, tr
     return c.finish(st, (out,))[0]
 
 
+@_layout_dispatch
 def rlscan_td_lambda(rewards, values, bootstrap, terminated=None, truncated=None, trunc_value=None,
                      *, gamma=0.99, lam=0.95, returns=None, stream=None, _tm=False):
     """TD(lambda) returns.  Returns the [N, T] returns."""
@@ -283,6 +310,7 @@ def rlscan_td_lambda(rewards, values, bootstrap, terminated=None, truncated=None
     return c.finish(st, (out,))[0]
 
 
+@_layout_dispatch
 def rlscan_discounted_return(rewards, bootstrap=None, terminated=None, truncated=None,
                              trunc_value=None, *, gamma=0.99, returns=None, stream=None, _tm=False):
     """Discounted returns (bootstrap optional).  Returns the [N, T] returns."""
@@ -301,6 +329,7 @@ def rlscan_discounted_return(rewards, bootstrap=None, terminated=None, truncated
     return c.finish(st, (out,))[0]
 
 
+@_layout_dispatch
 def rlscan_elig_trace(inputs, init_trace=None, terminated=None, truncated=None, *, gamma=0.99,
                       lam=0.95, traces=None, stream=None, _tm=False):
     """Accumulating eligibility traces (forward in time).  Returns the [N, T] traces."""
@@ -318,6 +347,7 @@ def rlscan_elig_trace(inputs, init_trace=None, terminated=None, truncated=None, 
     return c.finish(st, (out,))[0]
 
 
+@_layout_dispatch
 def rlscan_episodic_prefix_sum(x, terminated=None, truncated=None, *, out=None, stream=None, _tm=False):
     """Episodic inclusive prefix sums of int32 values.  Returns the [N, T] int32 sums."""
     name = "rlscan_episodic_prefix_sum_tm" if _tm else "rlscan_episodic_prefix_sum"
@@ -333,6 +363,7 @@ def rlscan_episodic_prefix_sum(x, terminated=None, truncated=None, *, out=None, 
     return c.finish(st, (o,))[0]
 
 
+@_layout_dispatch
 def rlscan_affine_scan(a, b, reset=None, init=None, *, reverse=False, x=None, stream=None, _tm=False):
     """Generic affine scan x_t = b_t + a_t x_prev along T (backward when
     `reverse`), x_prev = init[n] at the row's first step, x_t = b_t where

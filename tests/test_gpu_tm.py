@@ -217,3 +217,25 @@ def test_time_major_plan_shapes():
         info = slr.rlscan_query_plan_tm("gae", 1000, T)
         assert info["lookback"] == 0
         assert info["chunks"] == -(-1000 // (256 // slices))
+
+
+@pytest.mark.parametrize("est", TM_ESTIMATORS + ("affine_scan",))
+def test_transposed_views_take_the_time_major_kernel(est):
+    # [N, T] views of time-major [T, N] storage (buf.T) go to the time-major
+    # kernel without a copy; results come back as [N, T] views.
+    N, T = 96, 700
+    d = inputs(est, N, T, seed=3800)
+    s = f32_scalars(est, dict(synthetic.SCALARS.get(est, {})))
+    dt = transpose(d)
+    tv = {k: None if v is None else (torch.from_numpy(np.ascontiguousarray(v)).cuda() if k in PER_ENV
+                                     else torch.from_numpy(np.ascontiguousarray(v)).cuda().T)
+          for k, v in dt.items()}
+    import tests.util as U
+    t_orig = U.to_dev
+    U.to_dev = lambda dd, device="cuda": tv  # noqa: E731  (gpu_run takes the prepared views)
+    try:
+        got = U.gpu_run(est, d, **s)
+    finally:
+        U.to_dev = t_orig
+    ref = oracle_run(est, d, **s)
+    assert_parity(est, got, ref, what="transposed views")

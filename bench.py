@@ -42,13 +42,14 @@ DEFAULT_WORKLOAD = "sweep_4096xT"
 
 # Bytes per env-step each estimator must move at minimum (mandatory inputs
 # read once, outputs written once): fp32/int32 = 4 B, flags = 1 B.
-def algorithmic_bytes(est: str, d: dict) -> int:
+def algorithmic_bytes(est: str, d: dict, real_bytes: int = 4) -> int:
     """Strict algorithmic HBM bytes of one call on inputs `d`.
 
     Per-step arrays count their full size; `truncated` adds its flag bytes and
     `trunc_value` is counted only where truncated (one 32-byte sector each);
-    per-row arrays (bootstrap, init_trace) count 4 B per row; every output
-    counts 4 B per step."""
+    per-row arrays (bootstrap, init_trace) count one element per row; every
+    output counts one element per step.  `real_bytes` is the size of a real
+    element: 4 (fp32), or 2 for bf16 I/O."""
     if est == "affine_scan":  # a, b, reset flags, init per row, one output
         N, T = d["a"].shape
         return int(8 * N * T + (N * T if d.get("reset") is not None else 0)
@@ -66,7 +67,8 @@ def algorithmic_bytes(est: str, d: dict) -> int:
         "elig_trace": ("inputs",), "episodic_prefix_sum": ("x",),
         "retrace": ("mu_a", "actions", "rewards"),
     }[est]
-    b = sum(4 * nt for k in per_step_in)
+    rb = real_bytes
+    b = sum((4 if k == "actions" else rb) * nt for k in per_step_in)
     if est == "retrace":
         b += 2 * 4 * nt * A  # q and pi
     if d.get("terminated") is not None:
@@ -77,9 +79,9 @@ def algorithmic_bytes(est: str, d: dict) -> int:
             b += 32 * int(np.count_nonzero(d["truncated"]))
     for k in ("bootstrap", "init_trace"):
         if d.get(k) is not None:
-            b += 4 * N
+            b += rb * N
     n_out = {"gae": 2, "vtrace": 2}.get(est, 1)
-    b += 4 * nt * n_out
+    b += (4 if est == "episodic_prefix_sum" else rb) * nt * n_out
     return int(b)
 
 
@@ -220,6 +222,13 @@ def time_major(workload: str) -> bool:
     return synthetic.WORKLOADS[workload].get("layout") == "time_major"
 
 
+def bf16_io(workload: str) -> bool:
+    return synthetic.WORKLOADS[workload].get("io") == "bf16"
+
+
+REAL_KEYS = ("rewards", "values", "bootstrap", "trunc_value")  # the arrays bf16 I/O stores as bfloat16
+
+
 def call_arrays(est, d, tm):
     """The call's input arrays in argument order, time-major when `tm`."""
     dd = synthetic.to_time_major(d) if tm else d
@@ -233,21 +242,27 @@ def call_plan(slr, est, d, T, tm):
 
 
 class DeviceCall:
-    def __init__(self, est, T, d, device, tm=False):
+    def __init__(self, est, T, d, device, tm=False, bf16=False):
         import torch
-        self.est, self.T, self.tm = est, T, tm
-        self.inputs = [None if a is None else torch.from_numpy(a).to(device) for a in call_arrays(est, d, tm)]
+        self.est, self.T, self.tm, self.bf16 = est, T, tm, bf16
+        self.inputs = []
+        for k, a in zip(ARG_ORDER[est], call_arrays(est, d, tm)):
+            t = None if a is None else torch.from_numpy(a).to(device)
+            if t is not None and bf16 and k in REAL_KEYS:
+                t = t.to(torch.bfloat16)
+            self.inputs.append(t)
         shape = d["q"].shape[:2] if est == "retrace" else d[ARG_ORDER[est][0]].shape
         shape = tuple(shape[::-1]) if tm else tuple(shape)
-        dt = torch.int32 if est == "episodic_prefix_sum" else torch.float32
+        dt = torch.int32 if est == "episodic_prefix_sum" else (torch.bfloat16 if bf16 else torch.float32)
         self.outs = {k: torch.empty(shape, dtype=dt, device=device) for k in OUT_KW[est]}
         self.scal = {} if est == "episodic_prefix_sum" else dict(synthetic.SCALARS[est])
         self.steps = int(np.prod(shape))
-        self.bytes = algorithmic_bytes(est, d)
+        self.bytes = algorithmic_bytes(est, d, 2 if bf16 else 4)
+        self.fn = f"rlscan_{est}{'_tm' if tm else ''}{'_bf16' if bf16 else ''}"
 
     def launch(self):
         import segmented_linear_recurrence_b200 as slr
-        getattr(slr, f"rlscan_{self.est}{'_tm' if self.tm else ''}")(*self.inputs, **self.scal, **self.outs)
+        getattr(slr, self.fn)(*self.inputs, **self.scal, **self.outs)
 
 
 def run_gpu(args, rank, world, local_rank):
@@ -264,7 +279,7 @@ def run_gpu(args, rank, world, local_rank):
 
     host_calls = workload_calls(args.workload, rank)
     tm = time_major(args.workload)
-    calls = [DeviceCall(est, T, d, device, tm) for est, T, d in host_calls]
+    calls = [DeviceCall(est, T, d, device, tm, bf16_io(args.workload)) for est, T, d in host_calls]
     steps_per_step = sum(c.steps for c in calls)
     launches_per_step = 0
     for est, T, d in host_calls:
@@ -404,14 +419,19 @@ def run_e2e(args, host_calls, device, world):
     import segmented_linear_recurrence_b200 as slr
     pinned = []
     h2d = d2h = 0
-    tm = time_major(args.workload)
+    tm, bf16 = time_major(args.workload), bf16_io(args.workload)
     for est, T, d in host_calls:
-        ins = [None if a is None else torch.from_numpy(a).pin_memory() for a in call_arrays(est, d, tm)]
+        ins = []
+        for k, a in zip(ARG_ORDER[est], call_arrays(est, d, tm)):
+            t = None if a is None else torch.from_numpy(a)
+            if t is not None and bf16 and k in REAL_KEYS:
+                t = t.to(torch.bfloat16)
+            ins.append(None if t is None else t.pin_memory())
         h2d += sum(x.numel() * x.element_size() for x in ins if x is not None)
         shape = d["q"].shape[:2] if est == "retrace" else d[ARG_ORDER[est][0]].shape
-        d2h += 4 * int(np.prod(shape)) * len(OUT_KW[est])
+        d2h += (2 if bf16 else 4) * int(np.prod(shape)) * len(OUT_KW[est])
         scal = {} if est == "episodic_prefix_sum" else dict(synthetic.SCALARS[est])
-        pinned.append((f"rlscan_{est}{'_tm' if tm else ''}", ins, scal))
+        pinned.append((f"rlscan_{est}{'_tm' if tm else ''}{'_bf16' if bf16 else ''}", ins, scal))
 
     def step():
         out = None
@@ -625,6 +645,8 @@ def main():
     achieved = de["bytes"] / (de["ms"] / 1000.0) / 1e9
     tm = time_major(args.workload)
     dom_kernel = f"tm_scan_kernel<{dom}>" if tm else ("retrace_kernel" if dom == "retrace" else f"scan_kernel<{dom}>")
+    if bf16_io(args.workload):
+        dom_kernel = f"scan_kernel<{dom}, bf16 I/O>"
     traffic = load_traffic(args.workload, dom)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -642,7 +664,8 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": res["warmup"], "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 I/O, f32 arithmetic" if bf16_io(args.workload) else "f32",
+        "data": "synthetic",
         "config": {"workload": args.workload, "estimators": list(w["estimators"]),
                    "N_envs_per_gpu": w["N"], "T": list(w["Ts"]), "p_term": w["p_term"],
                    "p_trunc": w["p_trunc"], "calls_per_step": len(calls),

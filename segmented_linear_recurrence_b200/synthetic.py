@@ -53,6 +53,9 @@ WORKLOADS = {
     # the generic affine scan (backward), resets at p_term
     "affine_4096xT": dict(index=5, N=4096, Ts=(512, 2048), estimators=("affine_scan",), p_term=0.01,
                           p_trunc=0.0),
+    # GAE with bfloat16 I/O (inputs rounded to bf16 on the device side)
+    "gae_bf16_4096xT": dict(index=7, N=4096, Ts=(512, 2048), estimators=("gae",), p_term=0.02, p_trunc=0.005,
+                            io="bf16"),
     # the sweep's estimators and the affine scan on time-major [T, N] buffers
     "tm_4096xT": dict(index=6, N=4096, Ts=(512, 2048),
                       estimators=("gae", "vtrace", "td_lambda", "discounted_return", "affine_scan"),

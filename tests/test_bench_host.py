@@ -24,6 +24,9 @@ def test_algorithmic_bytes_per_step():
     assert bench.algorithmic_bytes("discounted_return", d) == 9 * N * T + 4 * N
     d = synthetic.make_affine_inputs(N, T, seed=1)
     assert bench.algorithmic_bytes("affine_scan", d) == 13 * N * T + 4 * N
+    # bf16 I/O: r, v, adv, ret 2 B each, the flag 1 B, bootstrap 2 B per row
+    d = synthetic.make_inputs("gae", N, T, seed=1, p_term=0.01, p_trunc=0.0)
+    assert bench.algorithmic_bytes("gae", d, real_bytes=2) == 9 * N * T + 2 * N
 
 
 def test_time_major_call_arrays_are_transposes():

@@ -18,11 +18,13 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  * Layout.  Per-step arrays are row-major [N, T] with T contiguous (one row per
- *   environment, the pages' [num_envs, seq_len] tensors, Probleemstelling).
+ *   environment, the pages' [num_envs, seq_len] tensors, Probleemstelling),
+ *   except for the "_tm" entry points, which take them time-major [T, N].
  *   Retrace's q and pi are [N, T, A] with A contiguous.  Per-row arrays
  *   (bootstrap, init_trace) are [N].
- * Types.  Values are float32, integers and actions int32, flags uint8 with
- *   nonzero meaning true (the byte layout of torch.bool).
+ * Types.  Values are float32 (bfloat16 bit patterns for the "_bf16" entry
+ *   points), integers and actions int32, flags uint8 with nonzero meaning true
+ *   (the byte layout of torch.bool).
  * Pointers.  Every pointer is a device-accessible address (device, managed or
  *   mapped pinned host memory) on the current CUDA device.  Float and int32
  *   arrays must be 4-byte aligned.  32-byte alignment of every per-step array

@@ -260,3 +260,20 @@ def test_gae_bf16_argument_checks(L):
                              None) == INVALID  # odd address
     assert L.rlscan_gae_bf16(r, v, b, None, None, None, v, None, 4, 8, 0.99, 0.95, None) == OVERLAP
     assert L.rlscan_gae_bf16(r, v, b, None, None, None, o, None, 4, 8, float("inf"), 0.95, None) == INVALID
+
+
+def test_plain_c_program_uses_the_abi(tmp_path):
+    # The header is C99 and the library links from C: a C user exercises the
+    # device-free calls (version, strings, plans, options, argument checks).
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = os.path.join(ROOT, "tests", "c", "abi_smoke.c")
+    exe = tmp_path / "abi_smoke"
+    libdir = os.path.dirname(slr.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), src,
+                    "-L", libdir, "-l:librlscan.so", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out.stderr
+    assert "abi_smoke ok" in out.stdout

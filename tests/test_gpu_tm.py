@@ -226,16 +226,25 @@ def test_transposed_views_take_the_time_major_kernel(est):
     N, T = 96, 700
     d = inputs(est, N, T, seed=3800)
     s = f32_scalars(est, dict(synthetic.SCALARS.get(est, {})))
-    dt = transpose(d)
-    tv = {k: None if v is None else (torch.from_numpy(np.ascontiguousarray(v)).cuda() if k in PER_ENV
-                                     else torch.from_numpy(np.ascontiguousarray(v)).cuda().T)
-          for k, v in dt.items()}
-    import tests.util as U
-    t_orig = U.to_dev
-    U.to_dev = lambda dd, device="cuda": tv  # noqa: E731  (gpu_run takes the prepared views)
-    try:
-        got = U.gpu_run(est, d, **s)
-    finally:
-        U.to_dev = t_orig
-    ref = oracle_run(est, d, **s)
-    assert_parity(est, got, ref, what="transposed views")
+    views = {k: None if v is None else (torch.from_numpy(np.ascontiguousarray(v)).cuda() if k in PER_ENV
+                                        else torch.from_numpy(np.ascontiguousarray(v)).cuda().T)
+             for k, v in transpose(d).items()}
+    args = {"gae": ("rewards", "values", "bootstrap", "terminated", "truncated", "trunc_value"),
+            "vtrace": ("log_rhos", "rewards", "values", "bootstrap", "terminated", "truncated", "trunc_value"),
+            "td_lambda": ("rewards", "values", "bootstrap", "terminated", "truncated", "trunc_value"),
+            "discounted_return": ("rewards", "bootstrap", "terminated", "truncated", "trunc_value"),
+            "elig_trace": ("inputs", "init_trace", "terminated", "truncated"),
+            "episodic_prefix_sum": ("x", "terminated", "truncated"),
+            "affine_scan": ("a", "b", "reset", "init")}[est]
+    kw = {} if est == "episodic_prefix_sum" else dict(s)
+    if est == "affine_scan":
+        kw = {"reverse": bool(s.get("reverse", False))}
+    for k, v in views.items():
+        if k not in PER_ENV and v is not None:
+            assert not v.is_contiguous() and v.shape == (N, T)
+    res = getattr(slr, f"rlscan_{est}")(*[views.get(k) for k in args], **kw)
+    res = res if isinstance(res, tuple) else (res,)
+    for r in res:
+        assert r is None or (r.shape == (N, T) and r.t().is_contiguous())
+    got = tuple(None if r is None else r.cpu().numpy() for r in res)
+    assert_parity(est, got, oracle_run(est, d, **s), what="transposed views")

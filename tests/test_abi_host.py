@@ -277,3 +277,27 @@ def test_plain_c_program_uses_the_abi(tmp_path):
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0, out.stderr
     assert "abi_smoke ok" in out.stdout
+
+
+def test_layout_dispatch_decision():
+    # The binding sends [N, T] views of time-major storage to the "_tm" path
+    # and everything else to the row-major path (decided on the host).
+    import torch
+    from segmented_linear_recurrence_b200 import api
+    seen = []
+
+    def fake(*args, _tm=False, **kw):
+        seen.append((_tm, [tuple(a.shape) for a in args if isinstance(a, torch.Tensor)]))
+        first = next(a for a in args if isinstance(a, torch.Tensor) and a.dim() == 2)
+        return first.clone(), None
+
+    f = api._layout_dispatch(fake)
+    buf_tm = torch.zeros(7, 5)          # [T, N] storage
+    per_env = torch.zeros(5)
+    out, none = f(buf_tm.T, buf_tm.T, per_env)
+    assert seen[-1] == (True, [(7, 5), (7, 5), (5,)]) and none is None
+    assert out.shape == (5, 7) and out.t().is_contiguous()   # [N, T] view of a [T, N] result
+    f(torch.zeros(5, 7), torch.zeros(5, 7), per_env)         # row-major: untouched
+    assert seen[-1] == (False, [(5, 7), (5, 7), (5,)])
+    f(buf_tm.T, torch.zeros(5, 7), per_env)                  # mixed layouts: row-major path (which then rejects)
+    assert seen[-1][0] is False
